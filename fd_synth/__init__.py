@@ -1,0 +1,190 @@
+"""Seeded synthetic inputs for the FlashDecoder streaming step.
+
+This module is shared by the CPU oracle's tests and by the CUDA path's
+tests and benchmark. It holds workload shapes and random-number recipes
+only: none of the decoder's arithmetic lives here.
+
+Shapes follow the FlashDecoder paper (academ.us/article/2607.14898):
+latent frames z_t of shape [C'][H'][W'] (Sec. 3.1), an optional
+PixelUnshuffle x2 of the Wan2.1 latent (Sec. 4.3, "Generalization Across
+Latent Spaces"), L_frm tokens per frame (Sec. 3.2, Eq. 1), a Transformer of
+width D with N heads of size D_h and G key/value groups (Sec. 3.2, 4.5).
+
+Recipe (stands in for UltraVideo clips encoded by the Wan encoders and for
+trained weights, neither of which is available):
+  * weights of every Linear ~ N(0,1)/sqrt(fan_in), biases likewise;
+  * RMSNorm / KV-norm gains = 1 + 0.1 N(0,1);
+  * latents ~ N(0,1);
+  * torch CPU generator, seed 0 for weights, seed 1 for latents;
+  * bf16 configurations round weights and latents to bf16 (nearest even)
+    before anyone sees them, so the oracle and the CUDA path read identical
+    values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class FDConfig:
+    """One decoder configuration (paper notation in comments)."""
+    name: str
+    latent_ch: int        # C'
+    grid_h: int           # H' (latent grid)
+    grid_w: int           # W'
+    patch: int            # PixelUnshuffle factor p (1 or 2)
+    d_model: int          # D
+    n_heads: int          # N (query heads)
+    n_kv_heads: int       # G (key/value groups)
+    head_dim: int         # D_h
+    n_blocks: int
+    mlp_ratio: int
+    window: int           # W = number of PAST latent frames kept; ring has W+1 slots
+    out_ch: int           # C (pixel channels)
+    r_t: int              # temporal upsampling factor
+    px_per_token: int     # P: pixels per token side
+    kv_norm: int          # 1 = KV-norm on
+    dtype: str            # "f32" or "bf16" (compute/storage of the CUDA path)
+    frames: int           # T' of the workload
+    norm_eps: float = 1e-6
+    rope_theta: float = 10000.0
+
+    # ---- derived shapes (no arithmetic of the method) ----
+    @property
+    def tok_h(self) -> int:
+        return self.grid_h // self.patch
+
+    @property
+    def tok_w(self) -> int:
+        return self.grid_w // self.patch
+
+    @property
+    def L_frm(self) -> int:
+        return self.tok_h * self.tok_w
+
+    @property
+    def c_in(self) -> int:
+        return self.latent_ch * self.patch * self.patch
+
+    @property
+    def qkv_dim(self) -> int:
+        return (self.n_heads + 2 * self.n_kv_heads) * self.head_dim
+
+    @property
+    def d_ff(self) -> int:
+        return self.mlp_ratio * self.d_model
+
+    @property
+    def c_out(self) -> int:
+        return self.out_ch * self.r_t * self.px_per_token * self.px_per_token
+
+    @property
+    def out_shape(self):
+        return (self.out_ch, self.r_t, self.tok_h * self.px_per_token,
+                self.tok_w * self.px_per_token)
+
+    def replace(self, **kw) -> "FDConfig":
+        return dataclasses.replace(self, **kw)
+
+
+CONFIGS: Dict[str, FDConfig] = {
+    # tiny fp32: 16ch latent, 8x8 grid, patch 1 (64 tokens), 3 frames, d=64,
+    # 2 heads x 32, 2 blocks, W=2, 3ch x 4 frames x 8x8 px per token.
+    "tiny_fp32": FDConfig("tiny_fp32", 16, 8, 8, 1, 64, 2, 2, 32, 2, 4, 2,
+                          3, 4, 8, 1, "f32", 3),
+    # Wan2.1-shaped 480p: 16ch, 60x104 grid, patch 2 (1560 tokens), 21 frames.
+    "480p_wan21": FDConfig("480p_wan21", 16, 60, 104, 2, 1024, 16, 16, 64, 12,
+                           4, 2, 3, 4, 16, 1, "bf16", 21),
+    # Wan2.1-shaped 720p: 16ch, 90x160 grid, patch 2 (3600 tokens), 21 frames.
+    "720p_wan21": FDConfig("720p_wan21", 16, 90, 160, 2, 1024, 16, 16, 64, 12,
+                           4, 2, 3, 4, 16, 1, "bf16", 21),
+    # Wan2.2-shaped 1080p: 48ch, 68x120 grid (1088x1920 px), patch 1
+    # (8160 tokens), 7 frames, 16 blocks.
+    "1080p_wan22": FDConfig("1080p_wan22", 48, 68, 120, 1, 1024, 16, 16, 64,
+                            16, 4, 2, 3, 4, 16, 1, "bf16", 7),
+    # long-stream Wan2.2-shaped 720p: 48ch, 45x80 grid, patch 1 (3600 tokens),
+    # 200 frames, 16 blocks.
+    "long720p_wan22": FDConfig("long720p_wan22", 48, 45, 80, 1, 1024, 16, 16,
+                               64, 16, 4, 2, 3, 4, 16, 1, "bf16", 200),
+}
+
+
+def weight_names(cfg: FDConfig) -> List[str]:
+    """Flat list of weight tensor names in generation order."""
+    names = ["embed_w", "embed_b"]
+    for l in range(cfg.n_blocks):
+        names += [f"b{l}.norm1_g", f"b{l}.wqkv", f"b{l}.bqkv", f"b{l}.knorm_g",
+                  f"b{l}.vnorm_g", f"b{l}.wo", f"b{l}.bo", f"b{l}.norm2_g",
+                  f"b{l}.w1", f"b{l}.b1", f"b{l}.w2", f"b{l}.b2"]
+    names += ["final_g", "out_w", "out_b"]
+    return names
+
+
+def weight_shapes(cfg: FDConfig) -> Dict[str, tuple]:
+    """Shapes in PyTorch Linear layout ([out][in]) and the fan_in of each."""
+    D, Dh, H = cfg.d_model, cfg.head_dim, cfg.n_heads
+    s = {"embed_w": ((D, cfg.c_in), cfg.c_in), "embed_b": ((D,), cfg.c_in)}
+    for l in range(cfg.n_blocks):
+        s[f"b{l}.norm1_g"] = ((D,), None)
+        s[f"b{l}.wqkv"] = ((cfg.qkv_dim, D), D)
+        s[f"b{l}.bqkv"] = ((cfg.qkv_dim,), D)
+        s[f"b{l}.knorm_g"] = ((Dh,), None)
+        s[f"b{l}.vnorm_g"] = ((Dh,), None)
+        s[f"b{l}.wo"] = ((D, H * Dh), H * Dh)
+        s[f"b{l}.bo"] = ((D,), H * Dh)
+        s[f"b{l}.norm2_g"] = ((D,), None)
+        s[f"b{l}.w1"] = ((cfg.d_ff, D), D)
+        s[f"b{l}.b1"] = ((cfg.d_ff,), D)
+        s[f"b{l}.w2"] = ((D, cfg.d_ff), cfg.d_ff)
+        s[f"b{l}.b2"] = ((D,), cfg.d_ff)
+    s["final_g"] = ((D,), None)
+    s["out_w"] = ((cfg.c_out, D), D)
+    s["out_b"] = ((cfg.c_out,), D)
+    return s
+
+
+def _round(t: torch.Tensor, dtype: str) -> torch.Tensor:
+    if dtype == "bf16":
+        return t.to(torch.bfloat16).to(torch.float32)
+    return t
+
+
+def make_weights(cfg: FDConfig, seed: int = 0) -> Dict[str, np.ndarray]:
+    """Random-init weights (float32 numpy, bf16-representable for bf16 configs)."""
+    g = torch.Generator().manual_seed(seed)
+    shapes = weight_shapes(cfg)
+    out = {}
+    for name in weight_names(cfg):
+        shape, fan_in = shapes[name]
+        r = torch.randn(shape, generator=g, dtype=torch.float32)
+        if fan_in is None:          # a norm gain
+            t = 1.0 + 0.1 * r
+        else:
+            t = r / math.sqrt(fan_in)
+        out[name] = _round(t, cfg.dtype).numpy()
+    return out
+
+
+def make_latents(cfg: FDConfig, frames: int | None = None,
+                 seed: int = 1) -> np.ndarray:
+    """Latent video z[t][C'][H'][W'] (float32 numpy), N(0,1)."""
+    T = cfg.frames if frames is None else frames
+    g = torch.Generator().manual_seed(seed)
+    z = torch.randn((T, cfg.latent_ch, cfg.grid_h, cfg.grid_w), generator=g,
+                    dtype=torch.float32)
+    return _round(z, cfg.dtype).numpy()
+
+
+def perturb_frame(z: np.ndarray, t: int, seed: int = 7,
+                  dtype: str = "f32") -> np.ndarray:
+    """Copy of z with frame t replaced by fresh N(0,1) values."""
+    g = torch.Generator().manual_seed(seed)
+    out = z.copy()
+    r = torch.randn(z.shape[1:], generator=g, dtype=torch.float32)
+    out[t] = _round(r, dtype).numpy()
+    return out
