@@ -1,0 +1,197 @@
+/*
+ * flashdec.h — C ABI of the FlashDecoder streaming step on NVIDIA B200 (sm_100a).
+ *
+ * The operation. "FlashDecoder: Real-Time Latent-to-Pixel Streaming Decoder
+ * with Transformers" (academ.us/article/2607.14898), Sec. 3.3 "Frame-by-Frame
+ * Processing": a video's latent frames z_0 .. z_{T'-1} are decoded one at a
+ * time. For frame t the latent is projected to L_frm tokens (Eq. 1); each
+ * Transformer block computes new keys and values, appends them to a rolling
+ * cache and evicts the oldest frame (Eq. 2), and the frame's queries attend,
+ * with no mask, to every cached token. A final projection turns each token
+ * into r_t pixel frames of P x P pixels (Sec. 3.4, Step 3).
+ *
+ * Conventions of this library:
+ *   - W (fd_config.window) counts PAST latent frames. The cache keeps the
+ *     current frame plus W past frames, i.e. W+1 ring slots per block; frame t
+ *     is stored in slot t mod (W+1). While t < W only the t+1 frames that
+ *     exist are attended to (no padding).
+ *   - Every call enqueues work on a CUDA stream and returns at once. A handle
+ *     is not thread-safe; one handle decodes one video stream at a time.
+ *   - All functions return FD_OK (0) or a negative fd_status_t. The message
+ *     of the last failure on the calling thread is fd_last_error().
+ *   - The library never falls back to another implementation: it runs its
+ *     own sm_100a kernels or returns an error.
+ */
+#ifndef FLASHDEC_H
+#define FLASHDEC_H
+
+#include <stdint.h>
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FD_API __attribute__((visibility("default")))
+#else
+#define FD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fd_handle fd_handle;   /* opaque */
+
+typedef enum {
+  FD_OK = 0,
+  FD_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, bad size, bad config */
+  FD_ERR_UNSUPPORTED = -2,   /* valid config the kernels do not implement    */
+  FD_ERR_OOM = -3,           /* device allocation failed                      */
+  FD_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed             */
+  FD_ERR_TIMEOUT = -5,       /* a device-side wait ran out (see fd_status)    */
+  FD_ERR_BAD_HANDLE = -6     /* null, destroyed or foreign handle             */
+} fd_status_t;
+
+typedef enum { FD_F32 = 0, FD_BF16 = 1 } fd_dtype;
+
+/* Decoder shape. Paper notation in brackets. */
+typedef struct {
+  int32_t latent_ch;     /* [C'] latent channels                                  */
+  int32_t grid_h;        /* [H'] latent rows per frame                            */
+  int32_t grid_w;        /* [W'] latent columns per frame                         */
+  int32_t patch;         /* p in {1,2}: PixelUnshuffle of the latent (Sec. 4.3)   */
+  int32_t d_model;       /* [D]                                                   */
+  int32_t n_heads;       /* [N] query heads                                       */
+  int32_t n_kv_heads;    /* [G] key/value groups (GQA); must divide n_heads       */
+  int32_t head_dim;      /* [D_h]                                                 */
+  int32_t n_blocks;      /* Transformer blocks                                    */
+  int32_t mlp_ratio;     /* hidden width = mlp_ratio * D                          */
+  int32_t window;        /* W: past latent frames kept (ring of W+1 slots)        */
+  int32_t out_ch;        /* [C] pixel channels                                    */
+  int32_t r_t;           /* [r_t] pixel frames per latent frame                   */
+  int32_t px_per_token;  /* P: each token becomes a P x P pixel patch             */
+  int32_t kv_norm;       /* 1: RMSNorm keys and values per head (Sec. 3.2)        */
+  fd_dtype dtype;        /* FD_F32: fp32 throughout; FD_BF16: bf16 storage with
+                            fp32 accumulation, fp32 residual stream and norms     */
+  fd_dtype io_dtype;     /* element type of latent_frame and out_pixels           */
+  float norm_eps;        /* RMSNorm epsilon (1e-6)                                */
+  float rope_theta;      /* RoPE base (1e4)                                       */
+  int32_t kernel_timing; /* 1: bracket each kernel with CUDA events (for
+                            fd_last_step_kernel_ms); 0: off                       */
+} fd_config;
+
+/*
+ * Weights: HOST float32 arrays in PyTorch Linear layout [out][in]. Per-block
+ * entries are arrays of n_blocks pointers. fd_create copies everything; the
+ * caller may free the arrays when it returns. For FD_BF16 the library folds
+ * each RMSNorm gain into the Linear that follows it and rounds to bf16
+ * (nearest even).
+ *   embed_w [D][C' p^2], embed_b [D]                      (Eq. 1; channel
+ *            order of a token = (c, dy, dx), tokens in raster order)
+ *   norm1_g [D]; wqkv [(N+2G) D_h][D] rows ordered [Q heads | K heads |
+ *            V heads], bqkv [(N+2G) D_h]; knorm_g, vnorm_g [D_h] (ignored
+ *            when kv_norm = 0); wo [D][N D_h], bo [D]; norm2_g [D];
+ *            w1 [mlp_ratio D][D], b1; w2 [D][mlp_ratio D], b2 [D]
+ *   final_g [D]; out_w [C r_t P^2][D] with output channel order
+ *            (c, tau, dy, dx); out_b [C r_t P^2]
+ */
+typedef struct {
+  const float *embed_w, *embed_b;
+  const float *const *norm1_g, *const *wqkv, *const *bqkv;
+  const float *const *knorm_g, *const *vnorm_g;
+  const float *const *wo, *const *bo, *const *norm2_g;
+  const float *const *w1, *const *b1, *const *w2, *const *b2;
+  const float *final_g, *out_w, *out_b;
+} fd_weights;
+
+/*
+ * Create a decoder on the current CUDA device: validates cfg, uploads the
+ * weights, allocates the ring cache and all scratch once (nothing is
+ * allocated per frame), builds the per-frame CUDA graph and leaves the
+ * decoder reset (frame counter 0, cache zeroed). Synchronous.
+ * Errors: FD_ERR_INVALID_ARG (null pointers, inconsistent shapes),
+ * FD_ERR_UNSUPPORTED (e.g. head_dim not 32/64, patch not 1/2, bf16 with
+ * D or widths not multiples of 64), FD_ERR_OOM, FD_ERR_CUDA. On error *out
+ * is set to NULL and nothing is leaked.
+ */
+FD_API fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle** out);
+
+/*
+ * Start a new video: frame counter := 0 and every ring slot zeroed, enqueued
+ * on `stream` (a cudaStream_t; NULL = legacy default stream). Sec. 3.3: the
+ * cache only ever holds frames of the current video.
+ */
+FD_API fd_status_t fd_reset(fd_handle* h, void* stream);
+
+/*
+ * Decode the next latent frame ([FD] Sec. 3.3, steps (1)-(3), then the output
+ * projection): enqueue one replay of the per-frame CUDA graph on `stream`.
+ *   latent_frame: DEVICE pointer, [C'][H'][W'] contiguous, io_dtype, one frame
+ *                 of a batch-1 NCTHW latent.
+ *   out_pixels:   DEVICE pointer, [C][r_t][H'P/p][W'P/p] contiguous, io_dtype.
+ * Both are owned by the caller, must be 16-byte aligned and must stay valid
+ * until the work on `stream` completes. Returns before the work finishes.
+ * Frames must be fed strictly in order. Device-side failures are reported
+ * by fd_status, not here.
+ */
+FD_API fd_status_t fd_decode_frame(fd_handle* h, const void* latent_frame, void* out_pixels,
+                            void* stream);
+
+/*
+ * Same as fd_decode_frame with HOST buffers: copies the latent frame to the
+ * device, decodes it and copies the pixels back, all on `stream`.
+ * For truly asynchronous copies both buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister). `out_pixels` is complete once the
+ * stream has been synchronised.
+ */
+FD_API fd_status_t fd_decode_frame_host(fd_handle* h, const void* latent_frame_host,
+                                 void* out_pixels_host, void* stream);
+
+/* Free every device resource of the handle (synchronises the device first). */
+FD_API void fd_destroy(fd_handle* h);
+
+/*
+ * Sticky device-side status of the handle: FD_OK, or FD_ERR_TIMEOUT if a
+ * bounded wait inside a kernel ran out (the kernel then returned early and
+ * its outputs are invalid). Synchronises the handle's last stream.
+ */
+FD_API fd_status_t fd_status(fd_handle* h);
+
+/* Static description of a status code. */
+FD_API const char* fd_error_string(fd_status_t s);
+
+/* Message of the last failure on the calling thread ("" if none). */
+FD_API const char* fd_last_error(void);
+
+/* Number of frames decoded since the last reset (synchronises). */
+FD_API fd_status_t fd_frame_index(fd_handle* h, int64_t* t_out);
+
+/* Device bytes held by the handle (weights, ring cache, scratch, staging). */
+FD_API fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out);
+
+/* Bytes of the ring cache alone: n_blocks * 2 * G * (W+1) L_frm * D_h * elt. */
+FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
+
+/*
+ * Test/debug: copy ring slot `slot` of block `block` to host memory as fp32
+ * [G][L_frm][D_h]. kv = 0 reads keys (stored after KV-norm and RoPE at the
+ * frame's absolute index), kv = 1 reads values (after KV-norm). Synchronous.
+ */
+FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
+
+/*
+ * Kernel timing (requires cfg.kernel_timing = 1): waits for the last
+ * enqueued frame and writes the device time in ms of each kernel of that
+ * frame, in launch order, to ms_out[0 .. n-1] and its kernel kind to
+ * kind_out (see fd_kernel_kind). *n_out = number of kernels in one frame.
+ * Pass cap = 0 to query *n_out only.
+ */
+typedef enum {
+  FD_K_STEP_BEGIN = 0, FD_K_EMBED = 1, FD_K_QKV = 2, FD_K_ATTN = 3,
+  FD_K_OPROJ = 4, FD_K_MLP_UP = 5, FD_K_MLP_DOWN = 6, FD_K_FINAL = 7
+} fd_kernel_kind;
+FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out,
+                                   int32_t cap, int32_t* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHDEC_H */

@@ -1,0 +1,906 @@
+// fd_api.cu — host runtime and C ABI of the FlashDecoder streaming step.
+//
+// fd_create validates the configuration, packs the weights (RMSNorm gains
+// folded into the following Linear, bf16 rounding), allocates the ring cache
+// and every scratch buffer once, encodes the TMA tensor maps and builds one
+// CUDA graph of the whole per-frame step (paper Sec. 4.6: the per-frame pass
+// is a fixed, data-independent graph). fd_decode_frame replays that graph.
+//
+// Per-frame kernel sequence (bf16 configuration, all sm_100a):
+//   step_begin -> embed -> n_blocks x [QKV GEMM (+norm, KV-norm, RoPE, ring
+//   write) -> attention -> O-proj GEMM (+residual) -> MLP-up GEMM (+GELU) ->
+//   MLP-down GEMM (+residual)] -> final GEMM (+norm, unpatchify)
+// The fp32 configuration runs the same sequence with CUDA-core kernels.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "fd_attn_tc.cuh"
+#include "fd_gemm_tc.cuh"
+#include "fd_simt.cuh"
+
+using namespace fd;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fd_status_t fail(fd_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define FD_CUDA(call)                                                                     \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess) {                                                              \
+      cudaGetLastError();                                                                 \
+      return fail(e_ == cudaErrorMemoryAllocation ? FD_ERR_OOM : FD_ERR_CUDA, "%s: %s", #call, \
+                  cudaGetErrorString(e_));                                                \
+    }                                                                                     \
+  } while (0)
+
+#define FD_TRY(expr)                     \
+  do {                                   \
+    fd_status_t s_ = (expr);             \
+    if (s_ != FD_OK) return s_;          \
+  } while (0)
+
+constexpr uint32_t kMagic = 0xFDEC0DE5u;
+constexpr uint32_t kDead = 0xDEADFD00u;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+uint16_t f32_to_bf16_bits(float f) {        // round to nearest even
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u) return uint16_t((u >> 16) | ((u & 0xFFFF) ? 0x40 : 0));
+  const uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return uint16_t(u >> 16);
+}
+
+float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = uint32_t(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+fd_status_t get_encode() {
+  if (g_encode) return FD_OK;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  FD_CUDA(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q));
+  if (q != cudaDriverEntryPointSuccess || !fn)
+    return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return FD_OK;
+}
+
+// bf16 tensor map with 128-byte swizzle. dims/strides innermost first;
+// strides[i] is the byte pitch of dimension i+1.
+fd_status_t make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides, const uint32_t* box) {
+  FD_TRY(get_encode());
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+                        reinterpret_cast<const cuuint64_t*>(dims),
+                        reinterpret_cast<const cuuint64_t*>(strides),
+                        reinterpret_cast<const cuuint32_t*>(box), estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FD_OK;
+}
+
+// Row-major [rows][cols] bf16 matrix read in boxes of box_rows x 64.
+fd_status_t make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return make_tmap(m, base, 2, dims, strides, box);
+}
+
+struct KernelLaunch {
+  const void* func;
+  dim3 grid, block;
+  size_t smem;
+  int kind;
+};
+
+}  // namespace
+
+// ============================================================== the handle
+struct fd_handle {
+  uint32_t magic = kMagic;
+  fd_config cfg{};
+  int bf = 0;                       // 1: bf16 storage + tcgen05 kernels
+  int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
+  int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
+  size_t latent_elems = 0, out_elems = 0, io_elt = 0, elt = 0;
+
+  std::vector<void*> allocs;
+  size_t dev_bytes = 0, cache_bytes = 0;
+
+  float *embed_wT = nullptr, *embed_b = nullptr;
+  std::vector<void*> wqkv, wo, w1, w2;
+  std::vector<float*> bqkv, bo, b1, b2, gk, gv;
+  void* wout = nullptr;
+  float* bout = nullptr;
+  void *kc = nullptr, *vtc = nullptr;
+  float *x32 = nullptr, *ssq = nullptr;
+  void *xb = nullptr, *q = nullptr, *o = nullptr, *hb = nullptr;
+  float2 *rope_row = nullptr, *rope_col = nullptr;
+  long long* ctr = nullptr;
+  FrameState* fs = nullptr;
+  int* status = nullptr;
+  void *latent_stage = nullptr, *out_stage = nullptr;
+
+  // TMA maps (bf16 path)
+  CUtensorMap tm_xb{}, tm_o{}, tm_h{}, tm_q{}, tm_k{}, tm_v{}, tm_wout{};
+  std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_w1, tm_w2;
+
+  // graph
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaGraphNode_t last_node = nullptr;
+  cudaGraphNode_t embed_node = nullptr, final_node = nullptr;
+  KernelLaunch embed_launch{}, final_launch{};
+  EmbedParams embed_p{};
+  EpiParams final_p{};
+  int final_K = 0;
+  const void* cur_latent = nullptr;
+  void* cur_out = nullptr;
+  std::vector<cudaEvent_t> events;
+  std::vector<int> kinds;
+  cudaStream_t last_stream = nullptr;
+
+  // ---------------------------------------------------------------- memory
+  template <typename P>
+  fd_status_t alloc(P** p, size_t bytes) {
+    void* d = nullptr;
+    cudaError_t e = cudaMalloc(&d, bytes ? bytes : 16);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(FD_ERR_OOM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+    }
+    allocs.push_back(d);
+    dev_bytes += bytes;
+    *p = static_cast<P*>(d);
+    return FD_OK;
+  }
+  fd_status_t upload(void** dst, const void* src, size_t bytes) {
+    FD_TRY(alloc(dst, bytes));
+    FD_CUDA(cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice));
+    return FD_OK;
+  }
+  fd_status_t upload_f32(float** dst, const float* src, size_t n) {
+    void* d;
+    FD_TRY(upload(&d, src, n * 4));
+    *dst = static_cast<float*>(d);
+    return FD_OK;
+  }
+  // Weight [rows][cols] with optional per-column gain folded in, in storage type.
+  fd_status_t upload_w(void** dst, const float* w, size_t rows, size_t cols, const float* gain) {
+    if (bf) {
+      std::vector<uint16_t> tmp(rows * cols);
+      for (size_t r = 0; r < rows; ++r)
+        for (size_t c = 0; c < cols; ++c) {
+          const double v = double(w[r * cols + c]) * (gain ? double(gain[c]) : 1.0);
+          tmp[r * cols + c] = f32_to_bf16_bits(float(v));
+        }
+      return upload(dst, tmp.data(), tmp.size() * 2);
+    }
+    std::vector<float> tmp(rows * cols);
+    for (size_t r = 0; r < rows; ++r)
+      for (size_t c = 0; c < cols; ++c)
+        tmp[r * cols + c] = float(double(w[r * cols + c]) * (gain ? double(gain[c]) : 1.0));
+    return upload(dst, tmp.data(), tmp.size() * 4);
+  }
+
+  ~fd_handle() {
+    if (exec) cudaGraphExecDestroy(exec);
+    if (graph) cudaGraphDestroy(graph);
+    for (auto e : events) cudaEventDestroy(e);
+    for (void* p : allocs) cudaFree(p);
+  }
+
+  // ---------------------------------------------------------------- graph
+  fd_status_t add_event() {
+    cudaEvent_t ev;
+    FD_CUDA(cudaEventCreate(&ev));
+    events.push_back(ev);
+    cudaGraphNode_t n;
+    FD_CUDA(cudaGraphAddEventRecordNode(&n, graph, last_node ? &last_node : nullptr,
+                                        last_node ? 1 : 0, ev));
+    last_node = n;
+    return FD_OK;
+  }
+  fd_status_t add_kernel(const KernelLaunch& k, void** args, cudaGraphNode_t* out_node = nullptr) {
+    cudaKernelNodeParams np{};
+    np.func = const_cast<void*>(k.func);
+    np.gridDim = k.grid;
+    np.blockDim = k.block;
+    np.sharedMemBytes = unsigned(k.smem);
+    np.kernelParams = args;
+    cudaGraphNode_t n;
+    FD_CUDA(cudaGraphAddKernelNode(&n, graph, last_node ? &last_node : nullptr, last_node ? 1 : 0,
+                                   &np));
+    last_node = n;
+    if (out_node) *out_node = n;
+    kinds.push_back(k.kind);
+    if (cfg.kernel_timing) FD_TRY(add_event());
+    return FD_OK;
+  }
+
+  fd_status_t build_graph();
+  fd_status_t add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, const void* A,
+                       const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
+                       cudaGraphNode_t* node);
+  EpiParams base_epi() const;
+};
+
+namespace {
+
+bool valid_handle(const fd_handle* h) { return h && h->magic == kMagic; }
+
+template <int BN, int KIND>
+fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
+  constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  using S = TcGemmSmem<BN, STAGES>;
+  const void* f = reinterpret_cast<const void*>(&tc_gemm_kernel<BN, STAGES, KIND, 64>);
+  FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc));
+  const int tiles = ((M + 127) / 128) * (N / BN);
+  k->func = f;
+  k->grid = dim3(std::min(tiles, num_sms));
+  k->block = dim3(192);
+  k->smem = S::kAlloc;
+  return FD_OK;
+}
+
+template <int KIND>
+fd_status_t tc_gemm_pick(int M, int N, int num_sms, int* bn, KernelLaunch* k) {
+  if (N % 256 == 0) { *bn = 256; return tc_gemm_launch<256, KIND>(M, N, num_sms, k); }
+  if (N % 128 == 0) { *bn = 128; return tc_gemm_launch<128, KIND>(M, N, num_sms, k); }
+  *bn = 64;
+  return tc_gemm_launch<64, KIND>(M, N, num_sms, k);
+}
+
+template <int KIND>
+const void* simt_gemm_fn(int dh) {
+  return dh == 32 ? reinterpret_cast<const void*>(&simt_gemm_kernel<KIND, 32>)
+                  : reinterpret_cast<const void*>(&simt_gemm_kernel<KIND, 64>);
+}
+
+}  // namespace
+
+EpiParams fd_handle::base_epi() const {
+  EpiParams e{};
+  e.M = L;
+  e.ssq = ssq;
+  e.ssq_parts = cfg.d_model / 32;
+  e.inv_d = 1.f / float(cfg.d_model);
+  e.eps = cfg.norm_eps;
+  e.x32 = x32;
+  e.xb = xb;
+  e.ssq_out = ssq;
+  e.D = cfg.d_model;
+  e.q = q;
+  e.H = cfg.n_heads;
+  e.G = cfg.n_kv_heads;
+  e.Dh = cfg.head_dim;
+  e.kv_rows = kv_rows;
+  e.vt_pitch = vt_pitch;
+  e.kv_norm = cfg.kv_norm;
+  e.fs = fs;
+  e.rope_row = rope_row;
+  e.rope_col = rope_col;
+  e.tok_w = tok_w;
+  e.tok_h = tok_h;
+  e.P = cfg.px_per_token;
+  e.out_bf16 = cfg.io_dtype == FD_BF16;
+  return e;
+}
+
+// Kernel arguments must outlive the graph's construction; cudaGraphAddKernelNode
+// copies the pointed-to values, so stack storage inside one call suffices.
+fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, const void* A,
+                                const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
+                                cudaGraphNode_t* node) {
+  ep.N = N;
+  KernelLaunch k{};
+  if (bf) {
+    int bn = 0;
+    switch (kind) {
+      case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(L, N, num_sms, &bn, &k)); break;
+      case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(L, N, num_sms, &bn, &k)); break;
+      case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(L, N, num_sms, &bn, &k)); break;
+      default: FD_TRY(tc_gemm_pick<EPI_FINAL>(L, N, num_sms, &bn, &k)); break;
+    }
+    CUtensorMap a = tmA, b = tmB;
+    int kk = K;
+    int* st = status;
+    void* args[] = {&a, &b, &kk, &ep, &st};
+    k.kind = fd_kind;
+    return add_kernel(k, args, node);
+  }
+  switch (kind) {
+    case EPI_QKV: k.func = simt_gemm_fn<EPI_QKV>(cfg.head_dim); break;
+    case EPI_RESID: k.func = simt_gemm_fn<EPI_RESID>(cfg.head_dim); break;
+    case EPI_GELU: k.func = simt_gemm_fn<EPI_GELU>(cfg.head_dim); break;
+    default: k.func = simt_gemm_fn<EPI_FINAL>(cfg.head_dim); break;
+  }
+  k.grid = dim3((L + 127) / 128, N / 64);
+  k.block = dim3(128);
+  k.smem = 0;
+  k.kind = fd_kind;
+  const float* a = static_cast<const float*>(A);
+  const float* b = static_cast<const float*>(B);
+  int kk = K;
+  void* args[] = {&a, &b, &kk, &ep};
+  return add_kernel(k, args, node);
+}
+
+fd_status_t fd_handle::build_graph() {
+  FD_CUDA(cudaGraphCreate(&graph, 0));
+  last_node = nullptr;
+  if (cfg.kernel_timing) FD_TRY(add_event());
+
+  // step_begin
+  {
+    KernelLaunch k{reinterpret_cast<const void*>(&step_begin_kernel), dim3(1), dim3(32), 0,
+                   FD_K_STEP_BEGIN};
+    long long* c = ctr;
+    FrameState* f = fs;
+    int W = cfg.window, dh = cfg.head_dim;
+    float th = cfg.rope_theta;
+    void* args[] = {&c, &f, &W, &dh, &th};
+    FD_TRY(add_kernel(k, args));
+  }
+  // embed
+  {
+    embed_p.latent = latent_stage;
+    embed_p.latent_bf16 = cfg.io_dtype == FD_BF16;
+    embed_p.C = cfg.latent_ch;
+    embed_p.Hl = cfg.grid_h;
+    embed_p.Wl = cfg.grid_w;
+    embed_p.p = cfg.patch;
+    embed_p.tok_w = tok_w;
+    embed_p.L = L;
+    embed_p.c_in = c_in;
+    embed_p.wT = embed_wT;
+    embed_p.b = embed_b;
+    embed_p.D = cfg.d_model;
+    embed_p.x32 = x32;
+    embed_p.xb = xb;
+    embed_p.ssq = ssq;
+    const void* f = bf ? reinterpret_cast<const void*>(&embed_kernel<bf16>)
+                       : reinterpret_cast<const void*>(&embed_kernel<float>);
+    embed_launch = KernelLaunch{f, dim3((L + kEmbedTok - 1) / kEmbedTok), dim3(256),
+                                size_t(kEmbedTok) * c_in * 4, FD_K_EMBED};
+    void* args[] = {&embed_p};
+    FD_TRY(add_kernel(embed_launch, args, &embed_node));
+    cur_latent = latent_stage;
+  }
+  const int D = cfg.d_model, H = cfg.n_heads, Dh = cfg.head_dim;
+  for (int l = 0; l < cfg.n_blocks; ++l) {
+    // QKV + KV-norm + RoPE + ring write
+    EpiParams e = base_epi();
+    e.bias = bqkv[l];
+    e.kc = static_cast<char*>(kc) + size_t(l) * cfg.n_kv_heads * kv_rows * Dh * elt;
+    e.vtc = static_cast<char*>(vtc) + size_t(l) * cfg.n_kv_heads * Dh * vt_pitch * elt;
+    e.gk = gk[l];
+    e.gv = gv[l];
+    FD_TRY(add_gemm(EPI_QKV, FD_K_QKV, tm_xb, xb, bf ? tm_wqkv[l] : tm_xb, wqkv[l], qkv, D, e, nullptr));
+    // attention
+    if (bf) {
+      TcAttnParams ap{};
+      ap.o = o;
+      ap.L = L;
+      ap.H = H;
+      ap.G = cfg.n_kv_heads;
+      ap.layer = l;
+      ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
+      ap.fs = fs;
+      ap.status = status;
+      const void* f = reinterpret_cast<const void*>(&tc_attn_kernel);
+      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   TcAttnSmem::kAlloc));
+      KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(192), size_t(TcAttnSmem::kAlloc),
+                     FD_K_ATTN};
+      CUtensorMap a = tm_q, b = tm_k, c = tm_v;
+      void* args[] = {&a, &b, &c, &ap};
+      FD_TRY(add_kernel(k, args));
+    } else {
+      AttnParams ap{};
+      ap.q = q;
+      ap.kc = static_cast<char*>(kc) + size_t(l) * cfg.n_kv_heads * kv_rows * Dh * elt;
+      ap.vtc = static_cast<char*>(vtc) + size_t(l) * cfg.n_kv_heads * Dh * vt_pitch * elt;
+      ap.o = o;
+      ap.L = L;
+      ap.H = H;
+      ap.G = cfg.n_kv_heads;
+      ap.kv_rows = kv_rows;
+      ap.vt_pitch = vt_pitch;
+      ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
+      ap.fs = fs;
+      ap.status = status;
+      const void* f = Dh == 32 ? reinterpret_cast<const void*>(&simt_attn_kernel<32>)
+                               : reinterpret_cast<const void*>(&simt_attn_kernel<64>);
+      KernelLaunch k{f, dim3((L + 63) / 64, H), dim3(64), 0, FD_K_ATTN};
+      void* args[] = {&ap};
+      FD_TRY(add_kernel(k, args));
+    }
+    // output projection + residual
+    e = base_epi();
+    e.bias = bo[l];
+    FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[l] : tm_o, wo[l], D, H * Dh, e,
+                    nullptr));
+    // MLP up + GELU
+    e = base_epi();
+    e.bias = b1[l];
+    e.hout = hb;
+    FD_TRY(add_gemm(EPI_GELU, FD_K_MLP_UP, tm_xb, xb, bf ? tm_w1[l] : tm_xb, w1[l], dff, D, e,
+                    nullptr));
+    // MLP down + residual
+    e = base_epi();
+    e.bias = b2[l];
+    FD_TRY(add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h, hb, bf ? tm_w2[l] : tm_h, w2[l], D, dff, e,
+                    nullptr));
+  }
+  // final norm + projection + unpatchify
+  {
+    final_p = base_epi();
+    final_p.bias = bout;
+    final_p.out = out_stage;
+    final_K = D;
+    FD_TRY(add_gemm(EPI_FINAL, FD_K_FINAL, tm_xb, xb, bf ? tm_wout : tm_xb, wout, c_out, D,
+                    final_p, &final_node));
+    final_p.N = c_out;
+    cudaKernelNodeParams np{};
+    FD_CUDA(cudaGraphKernelNodeGetParams(final_node, &np));
+    final_launch = KernelLaunch{np.func, np.gridDim, np.blockDim, np.sharedMemBytes, FD_K_FINAL};
+    cur_out = out_stage;
+  }
+  FD_CUDA(cudaGraphInstantiate(&exec, graph, 0));
+  return FD_OK;
+}
+
+// ============================================================== C ABI
+namespace {
+
+fd_status_t validate(const fd_config* c) {
+  if (c->latent_ch <= 0 || c->grid_h <= 0 || c->grid_w <= 0 || c->d_model <= 0 ||
+      c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 || c->n_blocks <= 0 ||
+      c->mlp_ratio <= 0 || c->window < 0 || c->out_ch <= 0 || c->r_t <= 0 ||
+      c->px_per_token <= 0)
+    return fail(FD_ERR_INVALID_ARG, "config: every size must be positive (window >= 0)");
+  if (c->patch != 1 && c->patch != 2)
+    return fail(FD_ERR_UNSUPPORTED, "config: patch must be 1 or 2 (got %d)", c->patch);
+  if (c->grid_h % c->patch || c->grid_w % c->patch)
+    return fail(FD_ERR_INVALID_ARG, "config: latent grid %dx%d not divisible by patch %d",
+                c->grid_h, c->grid_w, c->patch);
+  if (c->n_heads % c->n_kv_heads)
+    return fail(FD_ERR_INVALID_ARG, "config: n_kv_heads (%d) must divide n_heads (%d)",
+                c->n_kv_heads, c->n_heads);
+  if (c->dtype != FD_F32 && c->dtype != FD_BF16)
+    return fail(FD_ERR_INVALID_ARG, "config: unknown dtype %d", int(c->dtype));
+  if (c->io_dtype != FD_F32 && c->io_dtype != FD_BF16)
+    return fail(FD_ERR_INVALID_ARG, "config: unknown io_dtype %d", int(c->io_dtype));
+  if (c->kv_norm != 0 && c->kv_norm != 1)
+    return fail(FD_ERR_INVALID_ARG, "config: kv_norm must be 0 or 1");
+  if (!(c->norm_eps > 0.f) || !(c->rope_theta > 1.f))
+    return fail(FD_ERR_INVALID_ARG, "config: norm_eps must be > 0 and rope_theta > 1");
+  if (c->px_per_token != 8 && c->px_per_token != 16)
+    return fail(FD_ERR_UNSUPPORTED, "config: px_per_token must be 8 or 16");
+  if (c->d_model % 64)
+    return fail(FD_ERR_UNSUPPORTED, "config: d_model must be a multiple of 64");
+  const int qkv = (c->n_heads + 2 * c->n_kv_heads) * c->head_dim;
+  if (c->dtype == FD_BF16) {
+    if (c->head_dim != 64)
+      return fail(FD_ERR_UNSUPPORTED, "config: bf16 kernels need head_dim 64 (got %d)",
+                  c->head_dim);
+  } else {
+    if (c->head_dim != 32 && c->head_dim != 64)
+      return fail(FD_ERR_UNSUPPORTED, "config: head_dim must be 32 or 64 (got %d)", c->head_dim);
+    if (qkv % 64 || (c->n_heads * c->head_dim) % 32)
+      return fail(FD_ERR_UNSUPPORTED, "config: (N+2G)*D_h must be a multiple of 64");
+  }
+  const long long L = (long long)(c->grid_h / c->patch) * (c->grid_w / c->patch);
+  if (L * (c->window + 1) > (1LL << 30))
+    return fail(FD_ERR_UNSUPPORTED, "config: window of %lld tokens is too large",
+                L * (c->window + 1));
+  if (c->kernel_timing != 0 && c->kernel_timing != 1)
+    return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0 or 1");
+  return FD_OK;
+}
+
+fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h) {
+  h->cfg = *cfg;
+  const fd_config& c = *cfg;
+  h->bf = c.dtype == FD_BF16;
+  h->elt = h->bf ? 2 : 4;
+  h->io_elt = c.io_dtype == FD_BF16 ? 2 : 4;
+  h->tok_h = c.grid_h / c.patch;
+  h->tok_w = c.grid_w / c.patch;
+  h->L = h->tok_h * h->tok_w;
+  h->c_in = c.latent_ch * c.patch * c.patch;
+  h->qkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  h->dff = c.mlp_ratio * c.d_model;
+  h->c_out = c.out_ch * c.r_t * c.px_per_token * c.px_per_token;
+  h->kv_rows = (c.window + 1) * h->L;
+  h->vt_pitch = int(round_up(size_t(h->kv_rows), 64));
+  h->out_h = h->tok_h * c.px_per_token;
+  h->out_w = h->tok_w * c.px_per_token;
+  h->latent_elems = size_t(c.latent_ch) * c.grid_h * c.grid_w;
+  h->out_elems = size_t(c.out_ch) * c.r_t * h->out_h * h->out_w;
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev));
+  int major = 0;
+  FD_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  FD_CUDA(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+  if (major != 10)
+    return fail(FD_ERR_UNSUPPORTED, "device compute capability %d.x: this library is built for sm_100a",
+                major);
+
+  const int D = c.d_model, H = c.n_heads, G = c.n_kv_heads, Dh = c.head_dim, NB = c.n_blocks;
+  // ---- weights
+  {
+    std::vector<float> wT(size_t(h->c_in) * D);
+    for (int d = 0; d < D; ++d)
+      for (int ch = 0; ch < h->c_in; ++ch) wT[size_t(ch) * D + d] = w->embed_w[size_t(d) * h->c_in + ch];
+    FD_TRY(h->upload_f32(&h->embed_wT, wT.data(), wT.size()));
+    FD_TRY(h->upload_f32(&h->embed_b, w->embed_b, D));
+  }
+  std::vector<float> ones(std::max(D, Dh), 1.f);
+  for (int l = 0; l < NB; ++l) {
+    void* p;
+    FD_TRY(h->upload_w(&p, w->wqkv[l], h->qkv, D, w->norm1_g[l])); h->wqkv.push_back(p);
+    FD_TRY(h->upload_w(&p, w->wo[l], D, size_t(H) * Dh, nullptr)); h->wo.push_back(p);
+    FD_TRY(h->upload_w(&p, w->w1[l], h->dff, D, w->norm2_g[l])); h->w1.push_back(p);
+    FD_TRY(h->upload_w(&p, w->w2[l], D, h->dff, nullptr)); h->w2.push_back(p);
+    float* f;
+    FD_TRY(h->upload_f32(&f, w->bqkv[l], h->qkv)); h->bqkv.push_back(f);
+    FD_TRY(h->upload_f32(&f, w->bo[l], D)); h->bo.push_back(f);
+    FD_TRY(h->upload_f32(&f, w->b1[l], h->dff)); h->b1.push_back(f);
+    FD_TRY(h->upload_f32(&f, w->b2[l], D)); h->b2.push_back(f);
+    FD_TRY(h->upload_f32(&f, c.kv_norm ? w->knorm_g[l] : ones.data(), Dh)); h->gk.push_back(f);
+    FD_TRY(h->upload_f32(&f, c.kv_norm ? w->vnorm_g[l] : ones.data(), Dh)); h->gv.push_back(f);
+  }
+  FD_TRY(h->upload_w(&h->wout, w->out_w, h->c_out, D, w->final_g));
+  FD_TRY(h->upload_f32(&h->bout, w->out_b, h->c_out));
+
+  // ---- ring cache: K [NB][G][(W+1)L][Dh], V^T [NB][G][Dh][vt_pitch]
+  const size_t k_bytes = size_t(NB) * G * h->kv_rows * Dh * h->elt;
+  const size_t v_bytes = size_t(NB) * G * Dh * h->vt_pitch * h->elt;
+  FD_TRY(h->alloc(&h->kc, k_bytes));
+  FD_TRY(h->alloc(&h->vtc, v_bytes));
+  h->cache_bytes = k_bytes + v_bytes;
+
+  // ---- scratch
+  const size_t L = h->L;
+  FD_TRY(h->alloc(&h->x32, L * D * 4));
+  FD_TRY(h->alloc(&h->xb, L * D * h->elt));
+  FD_TRY(h->alloc(&h->ssq, L * (D / 32) * 4));
+  FD_TRY(h->alloc(&h->q, size_t(H) * L * Dh * h->elt));
+  FD_TRY(h->alloc(&h->o, L * H * Dh * h->elt));
+  FD_TRY(h->alloc(&h->hb, L * h->dff * h->elt));
+  FD_TRY(h->alloc(&h->ctr, 64));
+  FD_TRY(h->alloc(&h->fs, sizeof(FrameState)));
+  FD_TRY(h->alloc(&h->status, 16));
+  FD_TRY(h->alloc(&h->latent_stage, round_up(h->latent_elems * h->io_elt, 256)));
+  FD_TRY(h->alloc(&h->out_stage, round_up(h->out_elems * h->io_elt, 256)));
+
+  // ---- spatial RoPE tables (fp64 angles): row part and column part,
+  // d_s = 3 D_h / 8 dims each, pair m at frequency theta^(-2m/d_s)
+  {
+    const int ds = 3 * Dh / 8;
+    std::vector<float2> rr(size_t(h->tok_h) * (ds / 2)), rc(size_t(h->tok_w) * (ds / 2));
+    for (int i = 0; i < h->tok_h; ++i)
+      for (int m = 0; m < ds / 2; ++m) {
+        const double a = i * std::pow(double(c.rope_theta), -2.0 * m / ds);
+        rr[size_t(i) * (ds / 2) + m] = make_float2(float(std::cos(a)), float(std::sin(a)));
+      }
+    for (int j = 0; j < h->tok_w; ++j)
+      for (int m = 0; m < ds / 2; ++m) {
+        const double a = j * std::pow(double(c.rope_theta), -2.0 * m / ds);
+        rc[size_t(j) * (ds / 2) + m] = make_float2(float(std::cos(a)), float(std::sin(a)));
+      }
+    void* p;
+    FD_TRY(h->upload(&p, rr.data(), rr.size() * sizeof(float2))); h->rope_row = static_cast<float2*>(p);
+    FD_TRY(h->upload(&p, rc.data(), rc.size() * sizeof(float2))); h->rope_col = static_cast<float2*>(p);
+  }
+
+  // ---- tensor maps (bf16 path)
+  if (h->bf) {
+    FD_TRY(make_tmap_2d(&h->tm_xb, h->xb, L, D, 128));
+    FD_TRY(make_tmap_2d(&h->tm_o, h->o, L, size_t(H) * Dh, 128));
+    FD_TRY(make_tmap_2d(&h->tm_h, h->hb, L, h->dff, 128));
+    auto bn_of = [](int N) { return N % 256 == 0 ? 256u : (N % 128 == 0 ? 128u : 64u); };
+    for (int l = 0; l < NB; ++l) {
+      CUtensorMap m;
+      FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(h->qkv))); h->tm_wqkv.push_back(m);
+      FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D))); h->tm_wo.push_back(m);
+      FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
+      FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+    }
+    FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, h->c_out, D, bn_of(h->c_out)));
+    {   // Q [H][L][64]: box 64 x 128 x 1
+      const uint64_t dims[3] = {64, L, uint64_t(H)};
+      const uint64_t str[2] = {64 * 2, L * 64 * 2};
+      const uint32_t box[3] = {64, 128, 1};
+      FD_TRY(make_tmap(&h->tm_q, h->q, 3, dims, str, box));
+    }
+    {   // K [NB*G][kv_rows][64]: box 64 x 128 x 1
+      const uint64_t dims[3] = {64, uint64_t(h->kv_rows), uint64_t(NB) * G};
+      const uint64_t str[2] = {64 * 2, uint64_t(h->kv_rows) * 64 * 2};
+      const uint32_t box[3] = {64, 128, 1};
+      FD_TRY(make_tmap(&h->tm_k, h->kc, 3, dims, str, box));
+    }
+    {   // V^T [NB*G][64][vt_pitch]: box 64 keys x 64 dims x 1
+      const uint64_t dims[3] = {uint64_t(h->vt_pitch), 64, uint64_t(NB) * G};
+      const uint64_t str[2] = {uint64_t(h->vt_pitch) * 2, uint64_t(h->vt_pitch) * 64 * 2};
+      const uint32_t box[3] = {64, 64, 1};
+      FD_TRY(make_tmap(&h->tm_v, h->vtc, 3, dims, str, box));
+    }
+  }
+
+  // ---- reset state, build the graph
+  FD_CUDA(cudaMemset(h->kc, 0, k_bytes));
+  FD_CUDA(cudaMemset(h->vtc, 0, v_bytes));
+  FD_CUDA(cudaMemset(h->ctr, 0, 64));
+  FD_CUDA(cudaMemset(h->status, 0, 16));
+  FD_CUDA(cudaMemset(h->fs, 0, sizeof(FrameState)));
+  FD_TRY(h->build_graph());
+  FD_CUDA(cudaDeviceSynchronize());
+  return FD_OK;
+}
+
+fd_status_t patch_io(fd_handle* h, const void* latent, void* out) {
+  if (latent != h->cur_latent) {
+    h->embed_p.latent = latent;
+    void* args[] = {&h->embed_p};
+    cudaKernelNodeParams np{};
+    np.func = const_cast<void*>(h->embed_launch.func);
+    np.gridDim = h->embed_launch.grid;
+    np.blockDim = h->embed_launch.block;
+    np.sharedMemBytes = unsigned(h->embed_launch.smem);
+    np.kernelParams = args;
+    FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, h->embed_node, &np));
+    h->cur_latent = latent;
+  }
+  if (out != h->cur_out) {
+    h->final_p.out = out;
+    cudaKernelNodeParams np{};
+    np.func = const_cast<void*>(h->final_launch.func);
+    np.gridDim = h->final_launch.grid;
+    np.blockDim = h->final_launch.block;
+    np.sharedMemBytes = unsigned(h->final_launch.smem);
+    if (h->bf) {
+      CUtensorMap a = h->tm_xb, b = h->tm_wout;
+      int K = h->final_K;
+      int* st = h->status;
+      void* args[] = {&a, &b, &K, &h->final_p, &st};
+      np.kernelParams = args;
+      FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, h->final_node, &np));
+    } else {
+      const float* a = static_cast<const float*>(h->xb);
+      const float* b = static_cast<const float*>(h->wout);
+      int K = h->final_K;
+      void* args[] = {&a, &b, &K, &h->final_p};
+      np.kernelParams = args;
+      FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, h->final_node, &np));
+    }
+    h->cur_out = out;
+  }
+  return FD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle** out) {
+  g_last_error.clear();
+  if (out) *out = nullptr;
+  if (!cfg || !weights || !out) return fail(FD_ERR_INVALID_ARG, "fd_create: null argument");
+  FD_TRY(validate(cfg));
+  const fd_weights* w = weights;
+  if (!w->embed_w || !w->embed_b || !w->norm1_g || !w->wqkv || !w->bqkv || !w->wo || !w->bo ||
+      !w->norm2_g || !w->w1 || !w->b1 || !w->w2 || !w->b2 || !w->final_g || !w->out_w ||
+      !w->out_b || (cfg->kv_norm && (!w->knorm_g || !w->vnorm_g)))
+    return fail(FD_ERR_INVALID_ARG, "fd_create: null weight pointer");
+  for (int l = 0; l < cfg->n_blocks; ++l)
+    if (!w->norm1_g[l] || !w->wqkv[l] || !w->bqkv[l] || !w->wo[l] || !w->bo[l] ||
+        !w->norm2_g[l] || !w->w1[l] || !w->b1[l] || !w->w2[l] || !w->b2[l] ||
+        (cfg->kv_norm && (!w->knorm_g[l] || !w->vnorm_g[l])))
+      return fail(FD_ERR_INVALID_ARG, "fd_create: null weight pointer in block %d", l);
+  fd_handle* h = new (std::nothrow) fd_handle();
+  if (!h) return fail(FD_ERR_OOM, "fd_create: host allocation failed");
+  const fd_status_t s = create_impl(cfg, weights, h);
+  if (s != FD_OK) {
+    cudaDeviceSynchronize();
+    cudaGetLastError();
+    delete h;
+    return s;
+  }
+  *out = h;
+  return FD_OK;
+}
+
+fd_status_t fd_reset(fd_handle* h, void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_reset: invalid handle");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_CUDA(cudaMemsetAsync(h->kc, 0, size_t(h->cfg.n_blocks) * h->cfg.n_kv_heads * h->kv_rows *
+                                        h->cfg.head_dim * h->elt, s));
+  FD_CUDA(cudaMemsetAsync(h->vtc, 0, size_t(h->cfg.n_blocks) * h->cfg.n_kv_heads *
+                                         h->cfg.head_dim * h->vt_pitch * h->elt, s));
+  FD_CUDA(cudaMemsetAsync(h->ctr, 0, 64, s));
+  FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
+  h->last_stream = s;
+  return FD_OK;
+}
+
+fd_status_t fd_decode_frame(fd_handle* h, const void* latent, void* out, void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame: invalid handle");
+  if (!latent || !out) return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: null buffer");
+  if ((reinterpret_cast<uintptr_t>(latent) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: buffers must be 16-byte aligned");
+  cudaPointerAttributes a{}, b{};
+  FD_CUDA(cudaPointerGetAttributes(&a, latent));
+  FD_CUDA(cudaPointerGetAttributes(&b, out));
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: latent_frame is not device memory");
+  if (b.type != cudaMemoryTypeDevice && b.type != cudaMemoryTypeManaged)
+    return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: out_pixels is not device memory");
+  FD_TRY(patch_io(h, latent, out));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_CUDA(cudaGraphLaunch(h->exec, s));
+  h->last_stream = s;
+  return FD_OK;
+}
+
+fd_status_t fd_decode_frame_host(fd_handle* h, const void* latent_host, void* out_host,
+                                 void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame_host: invalid handle");
+  if (!latent_host || !out_host) return fail(FD_ERR_INVALID_ARG, "fd_decode_frame_host: null buffer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_CUDA(cudaMemcpyAsync(h->latent_stage, latent_host, h->latent_elems * h->io_elt,
+                          cudaMemcpyHostToDevice, s));
+  FD_TRY(patch_io(h, h->latent_stage, h->out_stage));
+  FD_CUDA(cudaGraphLaunch(h->exec, s));
+  FD_CUDA(cudaMemcpyAsync(out_host, h->out_stage, h->out_elems * h->io_elt,
+                          cudaMemcpyDeviceToHost, s));
+  h->last_stream = s;
+  return FD_OK;
+}
+
+void fd_destroy(fd_handle* h) {
+  if (!valid_handle(h)) return;
+  cudaDeviceSynchronize();
+  h->magic = kDead;
+  delete h;
+}
+
+fd_status_t fd_status(fd_handle* h) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_status: invalid handle");
+  FD_CUDA(cudaStreamSynchronize(h->last_stream));
+  int st = 0;
+  FD_CUDA(cudaMemcpy(&st, h->status, 4, cudaMemcpyDeviceToHost));
+  if (st != 0) return fail(fd_status_t(st), "device reported status %d", st);
+  return FD_OK;
+}
+
+const char* fd_error_string(fd_status_t s) {
+  switch (s) {
+    case FD_OK: return "ok";
+    case FD_ERR_INVALID_ARG: return "invalid argument";
+    case FD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FD_ERR_OOM: return "out of device memory";
+    case FD_ERR_CUDA: return "CUDA error";
+    case FD_ERR_TIMEOUT: return "device-side wait timed out";
+    case FD_ERR_BAD_HANDLE: return "invalid handle";
+  }
+  return "unknown status";
+}
+
+const char* fd_last_error(void) { return g_last_error.c_str(); }
+
+fd_status_t fd_frame_index(fd_handle* h, int64_t* t_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_frame_index: invalid handle");
+  if (!t_out) return fail(FD_ERR_INVALID_ARG, "fd_frame_index: null output");
+  FD_CUDA(cudaStreamSynchronize(h->last_stream));
+  long long t = 0;
+  FD_CUDA(cudaMemcpy(&t, h->ctr, 8, cudaMemcpyDeviceToHost));
+  *t_out = t;
+  return FD_OK;
+}
+
+fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_device_bytes: invalid handle");
+  if (!bytes_out) return fail(FD_ERR_INVALID_ARG, "fd_device_bytes: null output");
+  *bytes_out = h->dev_bytes;
+  return FD_OK;
+}
+
+fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_cache_bytes: invalid handle");
+  if (!bytes_out) return fail(FD_ERR_INVALID_ARG, "fd_cache_bytes: null output");
+  *bytes_out = h->cache_bytes;
+  return FD_OK;
+}
+
+fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_read_slot: invalid handle");
+  const fd_config& c = h->cfg;
+  if (block < 0 || block >= c.n_blocks || slot < 0 || slot > c.window || (kv != 0 && kv != 1) ||
+      !host_dst)
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_read_slot: bad block/slot/kv/dst");
+  FD_CUDA(cudaDeviceSynchronize());
+  const int G = c.n_kv_heads, Dh = c.head_dim, L = h->L;
+  const size_t n = size_t(G) * L * Dh;
+  std::vector<uint8_t> raw;
+  if (kv == 0) {
+    raw.resize(n * h->elt);
+    for (int g = 0; g < G; ++g) {
+      const size_t src = ((size_t(block) * G + g) * h->kv_rows + size_t(slot) * L) * Dh * h->elt;
+      FD_CUDA(cudaMemcpy(raw.data() + size_t(g) * L * Dh * h->elt,
+                         static_cast<char*>(h->kc) + src, size_t(L) * Dh * h->elt,
+                         cudaMemcpyDeviceToHost));
+    }
+    for (size_t i = 0; i < n; ++i)
+      host_dst[i] = h->bf ? bf16_bits_to_f32(reinterpret_cast<uint16_t*>(raw.data())[i])
+                          : reinterpret_cast<float*>(raw.data())[i];
+  } else {
+    // V^T [G][Dh][pitch] -> [G][L][Dh]
+    std::vector<uint8_t> rows(size_t(L) * h->elt);
+    for (int g = 0; g < G; ++g)
+      for (int d = 0; d < Dh; ++d) {
+        const size_t src = ((size_t(block) * G + g) * Dh + d) * h->vt_pitch + size_t(slot) * L;
+        FD_CUDA(cudaMemcpy(rows.data(), static_cast<char*>(h->vtc) + src * h->elt,
+                           size_t(L) * h->elt, cudaMemcpyDeviceToHost));
+        for (int n2 = 0; n2 < L; ++n2)
+          host_dst[(size_t(g) * L + n2) * Dh + d] =
+              h->bf ? bf16_bits_to_f32(reinterpret_cast<uint16_t*>(rows.data())[n2])
+                    : reinterpret_cast<float*>(rows.data())[n2];
+      }
+  }
+  return FD_OK;
+}
+
+fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out, int32_t cap,
+                                   int32_t* n_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_last_step_kernel_ms: invalid handle");
+  if (!n_out) return fail(FD_ERR_INVALID_ARG, "fd_last_step_kernel_ms: null n_out");
+  const int n = int(h->kinds.size());
+  *n_out = n;
+  if (cap == 0) return FD_OK;
+  if (!h->cfg.kernel_timing)
+    return fail(FD_ERR_INVALID_ARG, "fd_last_step_kernel_ms: handle created with kernel_timing=0");
+  if (!ms_out || !kind_out || cap < n)
+    return fail(FD_ERR_INVALID_ARG, "fd_last_step_kernel_ms: output arrays too small");
+  FD_CUDA(cudaEventSynchronize(h->events.back()));
+  for (int i = 0; i < n; ++i) {
+    float ms = 0.f;
+    FD_CUDA(cudaEventElapsedTime(&ms, h->events[i], h->events[i + 1]));
+    ms_out[i] = ms;
+    kind_out[i] = h->kinds[i];
+  }
+  return FD_OK;
+}
+
+}  // extern "C"

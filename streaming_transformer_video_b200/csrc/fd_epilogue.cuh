@@ -1,0 +1,202 @@
+// fd_epilogue.cuh — fused GEMM epilogues of the FlashDecoder step.
+//
+// A GEMM thread owns one token row and 64 consecutive accumulator columns
+// (fp32). The epilogue finishes the layer's math on them in registers and
+// writes the result where the next kernel wants it:
+//   QKV    RMSNorm row scale + bias, KV-norm, 3D-RoPE, Q to its buffer and
+//          K/V into the frame's ring slot            (paper Sec. 3.2, 3.3, Eq. 2)
+//   RESID  residual add into the fp32 stream x, its storage-type copy and
+//          the per-32-column sums of squares the next RMSNorm needs
+//   GELU   RMSNorm row scale + bias + exact GELU -> MLP hidden
+//   FINAL  RMSNorm row scale + bias -> unpatchify scatter into NCTHW pixels
+//          (Sec. 3.4, Step 3: depth-to-space)
+//
+// RMSNorm fusion: the gain g is folded into the following weight matrix at
+// create time, so RMSNorm(x) W^T = diag(r) (x (W diag g)^T) with
+// r = 1/sqrt(mean(x^2) + eps). The producer of x emits sums of x^2 over each
+// 32-column chunk; the consumer adds them up per row (deterministic order).
+#pragma once
+
+#include "fd_common.cuh"
+
+namespace fd {
+
+enum EpiKind { EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2, EPI_FINAL = 3 };
+
+struct EpiParams {
+  int M;                 // rows (tokens of the frame)
+  int N;                 // GEMM output columns
+  const float* bias;     // [N]
+  // RMSNorm row scale (QKV, GELU, FINAL)
+  const float* ssq;      // [M][ssq_parts] sums of squares of x
+  int ssq_parts;
+  float inv_d;           // 1 / D
+  float eps;
+  // RESID
+  float* x32;            // [M][D] fp32 residual stream (updated in place)
+  void* xb;              // [M][D] storage-type copy (next GEMM's A operand)
+  float* ssq_out;        // [M][D/32]
+  int D;
+  // QKV
+  void* q;               // [H][M][Dh]
+  void* kc;              // this block's keys   [G][kv_rows][Dh]
+  void* vtc;             // this block's values [G][Dh][vt_pitch] (transposed)
+  int H, G, Dh;
+  int kv_rows;           // (W+1) * M
+  int vt_pitch;          // row pitch of the transposed values (elements)
+  const float* gk;       // [Dh] KV-norm gains
+  const float* gv;
+  int kv_norm;
+  const FrameState* fs;
+  const float2* rope_row;  // [tok_h][d_s/2] (cos, sin)
+  const float2* rope_col;  // [tok_w][d_s/2]
+  int tok_w;
+  // GELU
+  void* hout;            // [M][N]
+  // FINAL
+  void* out;             // [C][r_t][tok_h*P][tok_w*P]
+  int out_bf16;          // pixel element type
+  int P;                 // pixels per token side
+  int tok_h;
+};
+
+__device__ __forceinline__ float row_scale(const EpiParams& p, int row) {
+  const float* s = p.ssq + size_t(row) * p.ssq_parts;
+  float acc = 0.f;
+  for (int i = 0; i < p.ssq_parts; ++i) acc += s[i];
+  return rsqrtf(acc * p.inv_d + p.eps);
+}
+
+__device__ __forceinline__ float gelu_erf(float x) {
+  return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
+}
+
+// In-place 3D-RoPE of one head vector v[DH] of token `row`: pairs (2m, 2m+1)
+// of the temporal part [0, DH/4) rotate by the frame's angle, the row part
+// [DH/4, DH/4 + 3DH/8) by the token's grid row, the column part by its column.
+template <int DH>
+__device__ __forceinline__ void rope_head(float* v, int row, const EpiParams& p) {
+  constexpr int dt = DH / 4, ds = 3 * DH / 8;
+  const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
+  const float2* rr = p.rope_row + size_t(i) * (ds / 2);
+  const float2* rc = p.rope_col + size_t(j) * (ds / 2);
+#pragma unroll
+  for (int m = 0; m < dt / 2; ++m) {
+    const float2 cs = p.fs->rope_t[m];
+    const float a = v[2 * m], b = v[2 * m + 1];
+    v[2 * m] = a * cs.x - b * cs.y;
+    v[2 * m + 1] = a * cs.y + b * cs.x;
+  }
+#pragma unroll
+  for (int m = 0; m < ds / 2; ++m) {
+    const float2 cs = __ldg(rr + m);
+    float* w = v + dt + 2 * m;
+    const float a = w[0], b = w[1];
+    w[0] = a * cs.x - b * cs.y;
+    w[1] = a * cs.y + b * cs.x;
+  }
+#pragma unroll
+  for (int m = 0; m < ds / 2; ++m) {
+    const float2 cs = __ldg(rc + m);
+    float* w = v + dt + ds + 2 * m;
+    const float a = w[0], b = w[1];
+    w[0] = a * cs.x - b * cs.y;
+    w[1] = a * cs.y + b * cs.x;
+  }
+}
+
+template <int DH>
+__device__ __forceinline__ void rms_head(float* v, const float* g, float eps) {
+  float s = 0.f;
+#pragma unroll
+  for (int d = 0; d < DH; ++d) s += v[d] * v[d];
+  const float r = rsqrtf(s * (1.f / DH) + eps);
+#pragma unroll
+  for (int d = 0; d < DH; ++d) v[d] = v[d] * r * __ldg(g + d);
+}
+
+// acc[64]: columns col0 .. col0+63 of token `row` (row < M guaranteed).
+template <int KIND, typename T, int DH>
+__device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0, float* acc,
+                                           float rs) {
+  if constexpr (KIND == EPI_QKV) {
+#pragma unroll
+    for (int hh = 0; hh < 64 / DH; ++hh) {
+      float* v = acc + hh * DH;
+      const int col = col0 + hh * DH;
+      const int head = col / DH;
+#pragma unroll
+      for (int d = 0; d < DH; ++d) v[d] = v[d] * rs + __ldg(p.bias + col + d);
+      if (head < p.H) {                                   // query head
+        rope_head<DH>(v, row, p);
+        T* dst = static_cast<T*>(p.q) + (size_t(head) * p.M + row) * DH;
+        store_vec<T, DH>(dst, v);
+      } else if (head < p.H + p.G) {                      // key group
+        const int g = head - p.H;
+        if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
+        rope_head<DH>(v, row, p);
+        const int key = p.fs->slot * p.M + row;
+        T* dst = static_cast<T*>(p.kc) + (size_t(g) * p.kv_rows + key) * DH;
+        store_vec<T, DH>(dst, v);
+      } else {                                            // value group
+        const int g = head - p.H - p.G;
+        if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
+        const int key = p.fs->slot * p.M + row;
+        T* dst = static_cast<T*>(p.vtc) + size_t(g) * DH * p.vt_pitch + key;
+#pragma unroll
+        for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch] = from_f<T>(v[d]);
+      }
+    }
+  } else if constexpr (KIND == EPI_RESID) {
+    float* x = p.x32 + size_t(row) * p.D + col0;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+      float4 o = *reinterpret_cast<const float4*>(x + c);
+      o.x += acc[c + 0] + __ldg(p.bias + col0 + c + 0);
+      o.y += acc[c + 1] + __ldg(p.bias + col0 + c + 1);
+      o.z += acc[c + 2] + __ldg(p.bias + col0 + c + 2);
+      o.w += acc[c + 3] + __ldg(p.bias + col0 + c + 3);
+      *reinterpret_cast<float4*>(x + c) = o;
+      acc[c + 0] = o.x; acc[c + 1] = o.y; acc[c + 2] = o.z; acc[c + 3] = o.w;
+    }
+    store_vec<T, 64>(static_cast<T*>(p.xb) + size_t(row) * p.D + col0, acc);
+    const int parts = p.D / 32;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) s += acc[h * 32 + c] * acc[h * 32 + c];
+      p.ssq_out[size_t(row) * parts + col0 / 32 + h] = s;
+    }
+  } else if constexpr (KIND == EPI_GELU) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * rs + __ldg(p.bias + col0 + c));
+    store_vec<T, 64>(static_cast<T*>(p.hout) + size_t(row) * p.N + col0, acc);
+  } else {  // EPI_FINAL
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] = acc[c] * rs + __ldg(p.bias + col0 + c);
+    const int P = p.P;
+    const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
+    const size_t out_w = size_t(p.tok_w) * P;
+    const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
+    // 64 columns = 64/P output rows of P pixels each; column
+    // ((c*r_t + tau)*P + dy)*P + dx maps to frame (c, tau), pixel row i*P+dy.
+    for (int s = 0; s < 64; s += P) {
+      const int col = col0 + s;
+      const int ct = col / (P * P);                 // c*r_t + tau
+      const int dy = (col / P) % P;
+      const size_t off = size_t(ct) * plane + (size_t(i) * P + dy) * out_w + size_t(j) * P;
+      if (p.out_bf16) {
+        bf16* dst = static_cast<bf16*>(p.out) + off;
+        if (P == 16) store_vec<bf16, 16>(dst, acc + s);
+        else store_vec<bf16, 8>(dst, acc + s);
+      } else {
+        float* dst = static_cast<float*>(p.out) + off;
+        if (P == 16) store_vec<float, 16>(dst, acc + s);
+        else store_vec<float, 8>(dst, acc + s);
+      }
+    }
+  }
+}
+
+}  // namespace fd

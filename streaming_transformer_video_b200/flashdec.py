@@ -1,0 +1,247 @@
+"""ctypes binding of libflashdec.so (include/flashdec.h).
+
+Argument marshalling only: every step of the decoder runs in the library's
+CUDA kernels. PyTorch is used by callers for device memory and streams; this
+module takes raw pointers (tensor.data_ptr()) and CUDA stream handles.
+If the shared library is missing the import fails loudly: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflashdec.so")
+
+FD_OK, FD_ERR_INVALID_ARG, FD_ERR_UNSUPPORTED, FD_ERR_OOM = 0, -1, -2, -3
+FD_ERR_CUDA, FD_ERR_TIMEOUT, FD_ERR_BAD_HANDLE = -4, -5, -6
+FD_F32, FD_BF16 = 0, 1
+KERNEL_KINDS = ["step_begin", "embed", "qkv", "attn", "oproj", "mlp_up", "mlp_down", "final"]
+
+EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
+           "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
+           "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms"]
+
+
+class FDConfigC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "latent_ch", "grid_h", "grid_w", "patch", "d_model", "n_heads", "n_kv_heads",
+        "head_dim", "n_blocks", "mlp_ratio", "window", "out_ch", "r_t", "px_per_token",
+        "kv_norm", "dtype", "io_dtype")] + [
+        ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+        ("kernel_timing", ctypes.c_int32)]
+
+
+_PF = ctypes.POINTER(ctypes.c_float)
+_PPF = ctypes.POINTER(_PF)
+
+
+class FDWeightsC(ctypes.Structure):
+    _fields_ = [("embed_w", _PF), ("embed_b", _PF),
+                ("norm1_g", _PPF), ("wqkv", _PPF), ("bqkv", _PPF),
+                ("knorm_g", _PPF), ("vnorm_g", _PPF),
+                ("wo", _PPF), ("bo", _PPF), ("norm2_g", _PPF),
+                ("w1", _PPF), ("b1", _PPF), ("w2", _PPF), ("b2", _PPF),
+                ("final_g", _PF), ("out_w", _PF), ("out_b", _PF)]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"libflashdec.so not found at {path}; build it with "
+                          "`python -m streaming_transformer_video_b200.csrc.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.fd_create.argtypes = [ctypes.POINTER(FDConfigC), ctypes.POINTER(FDWeightsC),
+                              ctypes.POINTER(vp)]
+    lib.fd_reset.argtypes = [vp, vp]
+    lib.fd_decode_frame.argtypes = [vp, vp, vp, vp]
+    lib.fd_decode_frame_host.argtypes = [vp, vp, vp, vp]
+    lib.fd_destroy.argtypes = [vp]
+    lib.fd_destroy.restype = None
+    lib.fd_status.argtypes = [vp]
+    lib.fd_error_string.argtypes = [i32]
+    lib.fd_error_string.restype = ctypes.c_char_p
+    lib.fd_last_error.argtypes = []
+    lib.fd_last_error.restype = ctypes.c_char_p
+    lib.fd_frame_index.argtypes = [vp, ctypes.POINTER(i64)]
+    lib.fd_device_bytes.argtypes = [vp, ctypes.POINTER(sz)]
+    lib.fd_cache_bytes.argtypes = [vp, ctypes.POINTER(sz)]
+    lib.fd_debug_read_slot.argtypes = [vp, i32, i32, i32, _PF]
+    lib.fd_last_step_kernel_ms.argtypes = [vp, _PF, ctypes.POINTER(i32), i32,
+                                           ctypes.POINTER(i32)]
+    for name in EXPORTS:
+        if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
+            getattr(lib, name).restype = i32
+    return lib
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+class FDError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        L = lib()
+        msg = L.fd_last_error().decode() or L.fd_error_string(code).decode()
+        super().__init__(f"{where}: {L.fd_error_string(code).decode()} ({code}): {msg}")
+        self.code = code
+
+
+def _check(code: int, where: str):
+    if code != FD_OK:
+        raise FDError(code, where)
+
+
+def _dtype_code(s) -> int:
+    if s in ("bf16", FD_BF16):
+        return FD_BF16
+    if s in ("f32", "fp32", FD_F32):
+        return FD_F32
+    raise ValueError(f"unknown dtype {s!r}")
+
+
+def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
+    """fd_config from any object with the decoder's shape attributes."""
+    c = FDConfigC()
+    for n in ("latent_ch", "grid_h", "grid_w", "patch", "d_model", "n_heads", "n_kv_heads",
+              "head_dim", "n_blocks", "mlp_ratio", "window", "out_ch", "r_t", "px_per_token",
+              "kv_norm"):
+        setattr(c, n, int(getattr(cfg, n)))
+    c.dtype = _dtype_code(cfg.dtype)
+    c.io_dtype = _dtype_code(io_dtype if io_dtype is not None else cfg.dtype)
+    c.norm_eps = float(getattr(cfg, "norm_eps", 1e-6))
+    c.rope_theta = float(getattr(cfg, "rope_theta", 1e4))
+    c.kernel_timing = 1 if kernel_timing else 0
+    return c
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if hasattr(stream, "cuda_stream"):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+class FlashDecoder:
+    """One streaming decoder (one video at a time) on the current CUDA device.
+
+    weights: dict name -> float32 array in PyTorch Linear layout, names
+    "embed_w", "embed_b", "b{l}.norm1_g", "b{l}.wqkv", "b{l}.bqkv",
+    "b{l}.knorm_g", "b{l}.vnorm_g", "b{l}.wo", "b{l}.bo", "b{l}.norm2_g",
+    "b{l}.w1", "b{l}.b1", "b{l}.w2", "b{l}.b2", "final_g", "out_w", "out_b".
+    """
+
+    def __init__(self, cfg, weights: Dict[str, np.ndarray], io_dtype=None,
+                 kernel_timing: bool = False):
+        self._lib = lib()
+        self.cfg = cfg
+        self.c = make_config(cfg, io_dtype, kernel_timing)
+        keep: List[np.ndarray] = []
+
+        def fp(name):
+            a = np.ascontiguousarray(np.asarray(weights[name], dtype=np.float32))
+            keep.append(a)
+            return a.ctypes.data_as(_PF)
+
+        def per_block(key):
+            arr = (_PF * cfg.n_blocks)(*[fp(f"b{l}.{key}") for l in range(cfg.n_blocks)])
+            keep.append(arr)
+            return ctypes.cast(arr, _PPF)
+
+        w = FDWeightsC()
+        w.embed_w, w.embed_b = fp("embed_w"), fp("embed_b")
+        for key in ("norm1_g", "wqkv", "bqkv", "knorm_g", "vnorm_g", "wo", "bo", "norm2_g",
+                    "w1", "b1", "w2", "b2"):
+            setattr(w, key, per_block(key))
+        w.final_g, w.out_w, w.out_b = fp("final_g"), fp("out_w"), fp("out_b")
+        h = ctypes.c_void_p()
+        _check(self._lib.fd_create(ctypes.byref(self.c), ctypes.byref(w), ctypes.byref(h)),
+               "fd_create")
+        self.h = h
+        del keep
+
+    # ------------------------------------------------------------------
+    def close(self):
+        if getattr(self, "h", None):
+            self._lib.fd_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # ------------------------------------------------------------------
+    def reset(self, stream=None):
+        _check(self._lib.fd_reset(self.h, _stream_handle(stream)), "fd_reset")
+
+    def decode_frame(self, latent, out, stream=None):
+        """latent, out: CUDA tensors (or raw device pointers as int)."""
+        lp = latent.data_ptr() if hasattr(latent, "data_ptr") else int(latent)
+        op = out.data_ptr() if hasattr(out, "data_ptr") else int(out)
+        _check(self._lib.fd_decode_frame(self.h, ctypes.c_void_p(lp), ctypes.c_void_p(op),
+                                         _stream_handle(stream)), "fd_decode_frame")
+
+    def decode_frame_host(self, latent, out, stream=None):
+        """latent, out: host buffers (pinned tensors or numpy arrays)."""
+        lp = latent.data_ptr() if hasattr(latent, "data_ptr") else latent.ctypes.data
+        op = out.data_ptr() if hasattr(out, "data_ptr") else out.ctypes.data
+        _check(self._lib.fd_decode_frame_host(self.h, ctypes.c_void_p(lp), ctypes.c_void_p(op),
+                                              _stream_handle(stream)), "fd_decode_frame_host")
+
+    def status(self) -> int:
+        return int(self._lib.fd_status(self.h))
+
+    def frame_index(self) -> int:
+        t = ctypes.c_int64()
+        _check(self._lib.fd_frame_index(self.h, ctypes.byref(t)), "fd_frame_index")
+        return t.value
+
+    def device_bytes(self) -> int:
+        b = ctypes.c_size_t()
+        _check(self._lib.fd_device_bytes(self.h, ctypes.byref(b)), "fd_device_bytes")
+        return b.value
+
+    def cache_bytes(self) -> int:
+        b = ctypes.c_size_t()
+        _check(self._lib.fd_cache_bytes(self.h, ctypes.byref(b)), "fd_cache_bytes")
+        return b.value
+
+    def read_slot(self, block: int, slot: int, kv: int) -> np.ndarray:
+        """Ring slot contents as float32 [G][L_frm][D_h] (kv 0 = keys, 1 = values)."""
+        cfg = self.cfg
+        L = (cfg.grid_h // cfg.patch) * (cfg.grid_w // cfg.patch)
+        out = np.empty((cfg.n_kv_heads, L, cfg.head_dim), dtype=np.float32)
+        _check(self._lib.fd_debug_read_slot(self.h, block, slot, kv, out.ctypes.data_as(_PF)),
+               "fd_debug_read_slot")
+        return out
+
+    def kernel_ms(self) -> List[Tuple[str, float]]:
+        """(kind, ms) of every kernel of the last frame (kernel_timing=True)."""
+        n = ctypes.c_int32()
+        _check(self._lib.fd_last_step_kernel_ms(self.h, None, None, 0, ctypes.byref(n)),
+               "fd_last_step_kernel_ms")
+        ms = (ctypes.c_float * n.value)()
+        kinds = (ctypes.c_int32 * n.value)()
+        _check(self._lib.fd_last_step_kernel_ms(self.h, ms, kinds, n.value, ctypes.byref(n)),
+               "fd_last_step_kernel_ms")
+        return [(KERNEL_KINDS[kinds[i]], float(ms[i])) for i in range(n.value)]

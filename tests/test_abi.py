@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports every declared entry point, and its host
+logic (argument and configuration validation) works without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import fd_synth
+from streaming_transformer_video_b200 import flashdec as fdb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flashdec.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FD_API\s+[\w\s\*]+?\b(fd_\w+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = fdb.lib()
+    names = _declared()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(fdb.EXPORTS) == names
+    out = subprocess.run(["nm", "-D", "--defined-only", fdb.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r" T (fd_\w+)", out))
+    assert exported == set(names)
+
+
+def test_ctypes_structs_match_the_c_header(tmp_path):
+    # compile a probe against the header and compare sizes and offsets
+    probe = tmp_path / "probe.c"
+    fields = [f[0] for f in fdb.FDConfigC._fields_]
+    wfields = [f[0] for f in fdb.FDWeightsC._fields_]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "flashdec.h"',
+             'int main(void){', 'printf("%zu %zu\\n", sizeof(fd_config), sizeof(fd_weights));']
+    lines += [f'printf("%zu\\n", offsetof(fd_config, {f}));' for f in fields]
+    lines += [f'printf("%zu\\n", offsetof(fd_weights, {f}));' for f in wfields]
+    lines += ['return 0;}']
+    probe.write_text("\n".join(lines))
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(probe), "-o", str(exe)],
+                   check=True)
+    vals = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                           check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(fdb.FDConfigC)
+    assert vals[1] == ctypes.sizeof(fdb.FDWeightsC)
+    got = vals[2:]
+    want = [getattr(fdb.FDConfigC, f).offset for f in fields] + \
+           [getattr(fdb.FDWeightsC, f).offset for f in wfields]
+    assert got == want
+
+
+def test_error_strings():
+    lib = fdb.lib()
+    for code in range(0, -7, -1):
+        s = lib.fd_error_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.fd_error_string(-99).decode() == "unknown status"
+
+
+def _create(cfg_c):
+    lib = fdb.lib()
+    w = fdb.FDWeightsC()
+    h = ctypes.c_void_p()
+    return lib.fd_create(ctypes.byref(cfg_c), ctypes.byref(w), ctypes.byref(h)), h
+
+
+def test_create_rejects_bad_configs_before_touching_the_device():
+    base = fd_synth.CONFIGS["tiny_fp32"]
+    lib = fdb.lib()
+    h = ctypes.c_void_p(1234)
+    assert lib.fd_create(None, None, ctypes.byref(h)) == fdb.FD_ERR_INVALID_ARG
+    assert h.value is None
+    cases = [
+        (dict(patch=3), fdb.FD_ERR_UNSUPPORTED),
+        (dict(grid_h=7, patch=2), fdb.FD_ERR_INVALID_ARG),
+        (dict(n_heads=3, n_kv_heads=2), fdb.FD_ERR_INVALID_ARG),
+        (dict(d_model=0), fdb.FD_ERR_INVALID_ARG),
+        (dict(window=-1), fdb.FD_ERR_INVALID_ARG),
+        (dict(px_per_token=4), fdb.FD_ERR_UNSUPPORTED),
+        (dict(d_model=96), fdb.FD_ERR_UNSUPPORTED),
+        (dict(head_dim=48), fdb.FD_ERR_UNSUPPORTED),
+        (dict(dtype="bf16", head_dim=32), fdb.FD_ERR_UNSUPPORTED),
+    ]
+    for kw, code in cases:
+        c = fdb.make_config(base.replace(**kw))
+        s, _ = _create(c)
+        assert s == code, (kw, s, lib.fd_last_error())
+        assert lib.fd_last_error().decode()
+    # valid shape but null weights
+    s, _ = _create(fdb.make_config(base))
+    assert s == fdb.FD_ERR_INVALID_ARG
+
+
+def test_bad_handle_calls():
+    lib = fdb.lib()
+    t = ctypes.c_int64()
+    b = ctypes.c_size_t()
+    assert lib.fd_reset(None, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_decode_frame(None, None, None, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_decode_frame_host(None, None, None, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_status(None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_frame_index(None, ctypes.byref(t)) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_device_bytes(None, ctypes.byref(b)) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_cache_bytes(None, ctypes.byref(b)) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_read_slot(None, 0, 0, 0, None) == fdb.FD_ERR_BAD_HANDLE
+    # a pointer to memory that is not a handle (magic check)
+    junk = (ctypes.c_uint32 * 64)()
+    assert lib.fd_reset(ctypes.cast(junk, ctypes.c_void_p), None) == fdb.FD_ERR_BAD_HANDLE
+    lib.fd_destroy(None)
+    lib.fd_destroy(ctypes.cast(junk, ctypes.c_void_p))
