@@ -1,0 +1,399 @@
+"""Benchmark of the FlashDecoder streaming step on B200.
+
+One step = one latent frame through the whole per-frame step (embed, every
+block's QKV / attention / O-proj / MLP, final projection + unpatchify), i.e.
+one replay of the library's CUDA graph via fd_decode_frame. The warm-up
+steps also fill the rolling cache, so every timed step runs with the full
+(W+1)-frame window. Each latent frame yields r_t = 4 pixel frames.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+  python bench.py --impl reference ...   (the CPU oracle on a bounded sample)
+
+Rank 0 prints one JSON line. With N > 1 (torchrun) every rank decodes its
+own independent video on its own GPU (replicas: the step has no exchange),
+the timed region is bracketed by barriers and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import fd_synth  # noqa: E402
+
+METRIC = "decoded pixel frames/s at 1080p; p50 per-latent-frame latency; % of bf16 TC peak"
+UNIT = "pixel frames/s"
+DEFAULT_CONFIG = "1080p_wan22"
+
+# DRAM traffic of one attention launch (one block, full window) measured by
+# ncu (dram__bytes_read.sum + dram__bytes_write.sum), see
+# profiles/block_1080p_ncu_full.md. Keyed by the sha256 of the kernel source:
+# when the kernel changes the figure no longer applies and is reported as null.
+NCU_ATTN_TRAFFIC = {
+    ("1080p_wan22", "ded5840851c6f523af4e6d4203bc20b87cddffbec89453bc51c7c9d0b67dfcf4"):
+        117145856 + 11172608,
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def describe(cfg) -> str:
+    return (f"{cfg.name}: latent {cfg.latent_ch}ch {cfg.grid_h}x{cfg.grid_w}, patch {cfg.patch} "
+            f"({cfg.L_frm} tokens/frame), d={cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}, "
+            f"{cfg.n_blocks} blocks, MLP {cfg.mlp_ratio}x, W={cfg.window}; each latent frame -> "
+            f"{cfg.out_ch}x{cfg.r_t}x{cfg.out_shape[2]}x{cfg.out_shape[3]} px")
+
+
+def flops_per_frame(cfg, n_valid=None):
+    """Algorithmic FLOPs of one latent frame (2 per MAC). n_valid: frames in
+    the window (default: full, W+1)."""
+    L, D, nb = cfg.L_frm, cfg.d_model, cfg.n_blocks
+    nv = cfg.window + 1 if n_valid is None else n_valid
+    qkv = 2 * L * D * cfg.qkv_dim
+    oproj = 2 * L * cfg.n_heads * cfg.head_dim * D
+    mlp = 2 * 2 * L * D * cfg.d_ff
+    attn = 4 * L * (nv * L) * cfg.n_heads * cfg.head_dim
+    gemm = nb * (qkv + oproj + mlp) + 2 * L * cfg.c_in * D + 2 * L * D * cfg.c_out
+    return gemm + nb * attn, nb * attn
+
+
+def attn_flops_per_launch(cfg):
+    L = cfg.L_frm
+    return 4 * L * ((cfg.window + 1) * L) * cfg.n_heads * cfg.head_dim
+
+
+def file_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
+        load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": float(np.median(load)) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), world, local
+    return None, 0, 1, 0
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, v):
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, v):
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample_seconds(cfg, weights_1blk, z):
+    """Time the CPU oracle on a bounded sample: frames 0..W of a 1-block
+    decoder at the workload's full width (untimed set-up), then frame W+1
+    (full window) timed, plus the embedding and head timed separately.
+    Returns (seconds per latent frame of the full-depth decoder, detail)."""
+    import oracle
+    cfg1 = cfg.replace(n_blocks=1)
+    dec = oracle.OracleDecoder(cfg1, weights_1blk)
+    for t in range(cfg.window + 1):
+        dec.decode_frame(z[t])
+    t0 = time.perf_counter()
+    dec.decode_frame(z[cfg.window + 1])
+    t_one = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    x = dec.embed(z[0])
+    dec.head(x)
+    t_eh = time.perf_counter() - t0
+    t_block = max(t_one - t_eh, 1e-9)
+    per_frame = t_eh + cfg.n_blocks * t_block
+    return per_frame, dict(t_block_s=t_block, t_embed_head_s=t_eh)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    # the CPU oracle: rank 0 alone runs it; other ranks exit without work
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    cfg = fd_synth.CONFIGS[args.config]
+    w1 = fd_synth.make_weights(cfg.replace(n_blocks=1))
+    frames = args.warmup + args.steps + cfg.window + 2
+    z = fd_synth.make_latents(cfg, frames=frames)
+    import oracle
+    dec = oracle.OracleDecoder(cfg.replace(n_blocks=1), w1)
+    for t in range(cfg.window + 1):                     # fill the window (not a step)
+        dec.decode_frame(z[t])
+    t = cfg.window + 1
+    for _ in range(args.warmup):
+        dec.decode_frame(z[t]); t += 1
+    t0 = time.perf_counter()
+    dec.head(dec.embed(z[0]))
+    t_eh = time.perf_counter() - t0
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        dec.decode_frame(z[t]); t += 1
+        times.append(time.perf_counter() - t0)
+    t_block = max(float(np.mean(times)) - t_eh, 1e-9)
+    per_frame = t_eh + cfg.n_blocks * t_block
+    value = cfg.r_t / per_frame
+    sample = (f"each step: one full-window latent frame of a 1-block decoder at the workload's "
+              f"full width ({cfg.L_frm} tokens, {(cfg.window + 1) * cfg.L_frm}-token window); "
+              f"per-frame time = embed+head + {cfg.n_blocks} x block time")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_frame * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(cfg), "latent_frame_per_step": 1},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main arm
+def run_flashdec(args):
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder
+    dist, rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    cfg = fd_synth.CONFIGS[args.config]
+    td = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    weights = fd_synth.make_weights(cfg)
+    n_frames = args.warmup + args.steps
+    z = fd_synth.make_latents(cfg, frames=n_frames, seed=1 + rank)
+    dec = FlashDecoder(cfg, weights, kernel_timing=True)
+    stream = torch.cuda.Stream()
+    lat = torch.from_numpy(z).to(td).cuda()
+    outs = [torch.empty(cfg.out_shape, dtype=td, device="cuda") for _ in range(2)]
+    with torch.cuda.stream(stream):
+        dec.reset(stream)
+        for t in range(args.warmup):
+            dec.decode_frame(lat[t], outs[t % 2], stream)
+    stream.synchronize()
+    assert dec.status() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    kern = {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(dist)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        t = args.warmup + i
+        ev[i][0].record(stream)
+        dec.decode_frame(lat[t], outs[t % 2], stream)
+        ev[i][1].record(stream)
+        # per-kernel device times of this frame (CUDA events inside the graph)
+        for kind, ms in dec.kernel_ms():
+            kern.setdefault(kind, []).append(ms)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    clk = clocks.stop()
+    assert dec.status() == 0
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(dist, total_ms)
+    lat_ms = [a.elapsed_time(b) for a, b in ev]
+    frames_all = sum_over_ranks(dist, args.steps)
+    value = cfg.r_t * frames_all / (total_ms / 1e3)
+    kernels_per_frame = len(dec.kernel_ms())
+
+    # ---- end to end: host buffers through fd_decode_frame_host
+    lat_h = [torch.from_numpy(z[t]).to(td).pin_memory() for t in range(n_frames)]
+    out_h = torch.empty(cfg.out_shape, dtype=td).pin_memory()
+    e2e_steps = args.steps
+    dec2 = FlashDecoder(cfg, weights)
+    with torch.cuda.stream(stream):
+        dec2.reset(stream)
+        for t in range(args.warmup):
+            dec2.decode_frame_host(lat_h[t], out_h, stream)
+    stream.synchronize()
+    barrier(dist)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        dec2.decode_frame_host(lat_h[args.warmup + i], out_h, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    assert dec2.status() == 0
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1))
+    e2e_value = cfg.r_t * sum_over_ranks(dist, e2e_steps) / (e2e_ms / 1e3)
+    h2d = int(np.prod(z.shape[1:])) * (2 if td == torch.bfloat16 else 4)
+    d2h = int(np.prod(cfg.out_shape)) * (2 if td == torch.bfloat16 else 4)
+    dev_bytes = dec.device_bytes()
+    dec2.close()
+
+    # ---- roofline of the dominant kernel (attention) and of the whole step
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    attn_ms = float(np.mean(kern["attn"]))
+    attn_tf = attn_flops_per_launch(cfg) / (attn_ms * 1e-3) / 1e12
+    src = os.path.join(ROOT, "streaming_transformer_video_b200", "csrc", "fd_attn_tc.cuh")
+    traffic = NCU_ATTN_TRAFFIC.get((args.config, file_sha(src)))
+    step_flops, _ = flops_per_frame(cfg)
+    step_tf = step_flops / (total_ms / args.steps * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        w1 = {k: v for k, v in weights.items() if not k.startswith("b") or k.startswith("b0.")}
+        per_frame, detail = oracle_sample_seconds(cfg, w1, z)
+        cpu = {"value": cfg.r_t / per_frame, "unit": UNIT, "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": (f"frame {cfg.window + 1} (full {cfg.window + 1}-frame window) of a "
+                          f"1-block decoder at full width, after frames 0..{cfg.window} "
+                          f"untimed; per-frame time = embed+head ({detail['t_embed_head_s']:.2f} s)"
+                          f" + {cfg.n_blocks} x block ({detail['t_block_s']:.2f} s)")}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": describe(cfg), "latent_frame_per_step": 1,
+                   "replicas": world,
+                   "l2": "no flush: every step streams ~%.1f GB (weights + ring cache) > 126 MB L2"
+                         % (dev_bytes / 1e9)},
+        "p50_ms": float(np.percentile(lat_ms, 50)), "p99_ms": float(np.percentile(lat_ms, 99)),
+        "latency_ms_by_step": [round(x, 4) for x in lat_ms],
+        "tc_frac_step": step_tf / peak,
+        "step_tflops": step_tf,
+        "roofline": {"bound": "tensor", "kernel": "tc_attn_kernel", "achieved": attn_tf,
+                     "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
+                     "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"},
+        "kernels_ms": {k: float(np.mean(v)) for k, v in kern.items()},
+        "kernels_tflops": {},
+        "clocks": clk,
+        "gpu_launches": kernels_per_frame * args.steps,
+        "device_bytes": dev_bytes,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+    }
+    L, D = cfg.L_frm, cfg.d_model
+    per_kind_flops = {"qkv": 2 * L * D * cfg.qkv_dim, "oproj": 2 * L * cfg.n_heads * cfg.head_dim * D,
+                      "mlp_up": 2 * L * D * cfg.d_ff, "mlp_down": 2 * L * D * cfg.d_ff,
+                      "final": 2 * L * D * cfg.c_out, "attn": attn_flops_per_launch(cfg)}
+    for k, f in per_kind_flops.items():
+        if k in line["kernels_ms"]:
+            line["kernels_tflops"][k] = f / (line["kernels_ms"][k] * 1e-3) / 1e12
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    dec.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=14)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", default="flashdec", choices=["flashdec", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(fd_synth.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_flashdec(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
