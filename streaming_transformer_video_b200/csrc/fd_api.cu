@@ -417,10 +417,15 @@ fd_status_t fd_handle::build_graph() {
       ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
       ap.fs = fs;
       ap.status = status;
-      const void* f = reinterpret_cast<const void*>(&tc_attn_kernel);
-      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   TcAttnSmem::kAlloc));
-      KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(192), size_t(TcAttnSmem::kAlloc),
+      // two query tiles per CTA when that still gives at least one full wave
+      const bool two = ((L + 255) / 256) * H >= num_sms;
+      const void* f = two ? reinterpret_cast<const void*>(&tc_attn_kernel<2>)
+                          : reinterpret_cast<const void*>(&tc_attn_kernel<1>);
+      const int smem_bytes = two ? TcAttnSmem<2>::kAlloc : TcAttnSmem<1>::kAlloc;
+      const int threads = two ? TcAttnSmem<2>::kThreads : TcAttnSmem<1>::kThreads;
+      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes));
+      const int qrows = two ? 256 : 128;
+      KernelLaunch k{f, dim3((L + qrows - 1) / qrows, H), dim3(threads), size_t(smem_bytes),
                      FD_K_ATTN};
       CUtensorMap a = tm_q, b = tm_k, c = tm_v;
       void* args[] = {&a, &b, &c, &ap};

@@ -6,17 +6,19 @@
 // are always the contiguous range [0, n_valid*L) and softmax, being
 // invariant to the order of keys, needs no slot bookkeeping.
 //
-// One CTA = one head x 128 queries, 192 threads:
-//   warp 0      TMA: the Q tile once, then K (128 keys x 64) and the
-//               transposed V (64 x 128 keys, as two 64-key halves) per stage
-//   warp 1      TMEM allocator; lane 0 issues S_j = Q K_j^T into one of two
-//               TMEM S buffers, then O += P_{j-1} V_{j-1} (software pipelined
-//               so the tensor core works on S_j while the softmax runs on
-//               S_{j-1})
-//   warps 2..5  softmax, one query row per thread: S row from TMEM, base-2
-//               online softmax with lazy rescaling (O is rescaled in TMEM
-//               only when the running max grows by more than 2^8), P as bf16
-//               into a 128-byte-swizzled shared tile, final O / l to global
+// One CTA = one head x QT query tiles of 128 (QT = 1 or 2), sharing every
+// K/V stage between the tiles. Warps:
+//   0            TMA: the Q tiles once, then per stage K (128 keys x 64) and
+//                the transposed V (64 x 128 keys, two 64-key halves)
+//   1            TMEM allocator; lane 0 issues, per key tile j,
+//                S_t = Q_t K_j^T for every query tile t (SS form), then
+//                O_t += P_t V_{j-1} (TS form: P read from TMEM)
+//   2 .. 1+4*QT  softmax, one warpgroup per query tile, one query row per
+//                thread: S row from TMEM, base-2 online softmax with lazy
+//                rescaling (O is rescaled in TMEM only when the running max
+//                grows by more than 2^8), P packed to bf16 into TMEM
+// TMEM columns: S_t [128 t, 128 t + 128), O_t [256 + 64 t, +64),
+//               P_t [384 + 64 t, +64) (128 bf16 keys packed 2 per column).
 // Keys past n_valid*L inside the last tile get probability 0.
 #pragma once
 
@@ -33,23 +35,30 @@ struct TcAttnParams {
   int* status;
 };
 
-constexpr int kAttnStages = 3;
+template <int QT>
 struct TcAttnSmem {
-  static constexpr int kQ = 0;                       // 128 x 64 bf16 = 16 KB
-  static constexpr int kKV = 16384;                  // stages x (K 16 KB + V 16 KB)
+  static constexpr int kStages = QT == 2 ? 4 : 4;
+  static constexpr int kQ = 0;                                // QT x 16 KB
+  static constexpr int kKV = QT * 16384;                      // stages x (K 16 KB + V 16 KB)
   static constexpr int kKVStage = 32768;
-  static constexpr int kP = kKV + kAttnStages * kKVStage;   // 2 x 32 KB
-  static constexpr int kBar = kP + 2 * 32768;
-  // q_full, kv_full[ST], kv_empty[ST], s_full[2], s_free[2], p_full[2], p_free[2], o_final
-  static constexpr int kNumBars = 1 + 2 * kAttnStages + 8 + 1;
+  static constexpr int kBar = kKV + kStages * kKVStage;
+  // q_full, kv_full[ST], kv_empty[ST], s_full[2], s_free[2], p_full[2], p_free[2], o_final[2]
+  static constexpr int kNumBars = 1 + 2 * kStages + 10;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kThreads = 64 + 128 * QT;
 };
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -68,17 +77,28 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T (A: M rows in lanes, K packed 2 per column).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);      // a -> low half (lower k)
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(192, 1)
+template <int QT>
+__global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcAttnParams p) {
-  using S = TcAttnSmem;
-  constexpr int ST = kAttnStages;
-  constexpr uint32_t kTmemCols = 512;                  // S0 [0,128) S1 [128,256) O [256,320)
+  using S = TcAttnSmem<QT>;
+  constexpr int ST = S::kStages;
+  constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128);
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, 64);
 
@@ -94,11 +114,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* p_full = s_free + 2;
   uint64_t* p_free = p_full + 2;
   uint64_t* o_final = p_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 128, h = blockIdx.y;
+  const int q0 = blockIdx.x * (128 * QT), h = blockIdx.y;
   const int g = h / (p.H / p.G);
   const int lg = p.layer * p.G + g;
   const int n_keys = p.fs->n_valid * p.L;
@@ -107,11 +127,11 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1); mbar_init(&s_free[b], 128);
-      mbar_init(&p_full[b], 128); mbar_init(&p_free[b], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1); mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128); mbar_init(&p_free[t], 1);
+      mbar_init(&o_final[t], 1);
     }
-    mbar_init(o_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmQ); prefetch_tensormap(&tmK); prefetch_tensormap(&tmV);
@@ -121,16 +141,15 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_o = tmem_base + 256;
 
   if (warp == 0) {
     if (lane == 0) {                                       // ---- TMA producer
-      mbar_arrive_expect_tx(q_full, 16384);
-      tma_load_3d(smem + S::kQ, &tmQ, 0, q0, h, q_full);
+      mbar_arrive_expect_tx(q_full, QT * 16384);
+      for (int t = 0; t < QT; ++t)
+        tma_load_3d(smem + S::kQ + t * 16384, &tmQ, 0, q0 + t * 128, h, q_full);
       for (int j = 0; j < n_kt; ++j) {
         const int st = j % ST;
-        const uint32_t ph = (j / ST) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* kv = smem + S::kKV + st * S::kKVStage;
         mbar_arrive_expect_tx(&kv_full[st], S::kKVStage);
         tma_load_3d(kv, &tmK, 0, j * 128, lg, &kv_full[st]);
@@ -140,54 +159,66 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {                                       // ---- MMA issuer
-      const uint32_t sq = smem_u32(smem + S::kQ);
-      auto issue_pv = [&](int i) -> bool {
-        const int b = i & 1, st = i % ST;
-        if (!mbar_wait(&p_full[b], (i >> 1) & 1, abort_flag, p.status)) return false;
+      // O_t += P_t(i) V(i): A from TMEM (P_t), B = V^T halves in shared memory
+      auto issue_pv = [&](int t, int i) -> bool {
+        if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t sp = smem_u32(smem + S::kP + b * 32768);
-        const uint32_t sv = smem_u32(smem + S::kKV + st * S::kKVStage + 16384);
+        const uint32_t sv = smem_u32(smem + S::kKV + (i % ST) * S::kKVStage + 16384);
+        const uint32_t a_tm = tmem_base + 384 + 64 * t;
+        const uint32_t d_tm = tmem_base + 256 + 64 * t;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int half = k >> 2, kk = k & 3;
-          tc_mma_ss(tmem_o, sw128_desc(sp + half * 16384) + 2 * kk,
-                    sw128_desc(sv + half * 8192) + 2 * kk, kIdescO, (i | k) != 0);
-        }
-        tc_commit(&p_free[b]);
-        tc_commit(&kv_empty[st]);
+        for (int k = 0; k < 8; ++k)
+          tc_mma_ts(d_tm, a_tm + 8 * k, sw128_desc(sv + (k >> 2) * 8192) + 2 * (k & 3), kIdescO,
+                    (i | k) != 0);
+        tc_commit(&p_free[t]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < n_kt; ++j) {
-        const int st = j % ST, b = j & 1;
+        const int st = j % ST;
         if (!mbar_wait(&kv_full[st], (j / ST) & 1, abort_flag, p.status)) { ok = false; break; }
-        if (!mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t sk = smem_u32(smem + S::kKV + st * S::kKVStage);
+        for (int t = 0; t < QT; ++t) {
+          if (!mbar_wait(&s_free[t], (j & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sq = smem_u32(smem + S::kQ + t * 16384);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_ss(tmem_base + b * 128, sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k, kIdescS,
-                    k != 0);
-        tc_commit(&s_full[b]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+          for (int k = 0; k < 4; ++k)
+            tc_mma_ss(tmem_base + 128 * t, sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k, kIdescS,
+                      k != 0);
+          tc_commit(&s_full[t]);
+        }
+        if (!ok) break;
+        if (j >= 1) {
+          for (int t = 0; t < QT && ok; ++t) ok = issue_pv(t, j - 1);
+          if (ok) tc_commit(&kv_empty[(j - 1) % ST]);
+        }
       }
-      if (ok && issue_pv(n_kt - 1)) tc_commit(o_final);
+      if (ok) {
+        for (int t = 0; t < QT && ok; ++t) ok = issue_pv(t, n_kt - 1);
+        if (ok)
+          for (int t = 0; t < QT; ++t) tc_commit(&o_final[t]);
+      }
     }
-  } else {                                                 // ---- softmax warps 2..5
-    const int quarter = warp & 3;
+  } else {                                                 // ---- softmax warpgroups
+    const int t = (warp - 2) >> 2;                         // query tile of this warpgroup
+    const int quarter = warp & 3;                          // TMEM lanes 32*quarter ..
     const int r = quarter * 32 + lane;                     // query row within the tile
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t tm_s = tmem_base + lane_off + 128 * t;
+    const uint32_t tm_o = tmem_base + lane_off + 256 + 64 * t;
+    const uint32_t tm_p = tmem_base + lane_off + 384 + 64 * t;
+    const float sc = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait_warp(&s_full[b], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&s_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
       float x[128];
       {
         uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ta = tmem_base + lane_off + b * 128;
-        tmem_ld32(ta, r0); tmem_ld32(ta + 32, r1); tmem_ld32(ta + 64, r2); tmem_ld32(ta + 96, r3);
+        tmem_ld32(tm_s, r0); tmem_ld32(tm_s + 32, r1); tmem_ld32(tm_s + 64, r2);
+        tmem_ld32(tm_s + 96, r3);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -196,67 +227,86 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&s_free[b]);
+      mbar_arrive(&s_free[t]);
       const int valid = n_keys - j * 128;                  // keys of this tile in range
-      float mx = -INFINITY;
+      if (valid < 128) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = (c < valid) ? x[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < 128; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
       }
-      if (j == 0) {
-        m_ref = mx;
-      } else if (mx > m_ref + 8.f) {
-        // rescale O and l to the new reference max; O must hold P_{j-1} V_{j-1}
-        if (!mbar_wait_warp(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      // row max of the raw scores (the scale is positive)
+      float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
+      float m2 = max3(x[6], x[7], x[8]), m3 = max3(x[9], x[10], x[11]);
+#pragma unroll
+      for (int c = 12; c < 124; c += 8) {
+        m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]);
+        m2 = max3(m2, x[c + 4], x[c + 5]); m3 = max3(m3, x[c + 6], x[c + 7]);
+      }
+      m0 = max3(m0, x[124], x[125]); m1 = max3(m1, x[126], x[127]);
+      const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sc;
+      bool rescale = false;
+      if (j == 0) m_ref = mx;
+      else if (mx > m_ref + 8.f) rescale = true;
+      // P_t and O_t are free once the MMA of the previous tile has finished
+      if (j >= 1) {
+        if (!mbar_wait_warp(&p_free[t], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
-        const float corr = ex2(m_ref - mx);
-        m_ref = mx;
-        l *= corr;
+      }
+      const float corr = rescale ? ex2(m_ref - mx) : 1.f;
+      if (rescale) { m_ref = mx; l *= corr; }
+      // p = 2^(s * scale - m_ref), packed fp32 pairs; row sum in 4 partials
+      const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m_ref, -m_ref);
+      float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        float2 e0 = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nm2);
+        float2 e1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), sc2, nm2);
+        float2 e2 = __ffma2_rn(make_float2(x[c + 4], x[c + 5]), sc2, nm2);
+        float2 e3 = __ffma2_rn(make_float2(x[c + 6], x[c + 7]), sc2, nm2);
+        e0 = make_float2(ex2(e0.x), ex2(e0.y)); e1 = make_float2(ex2(e1.x), ex2(e1.y));
+        e2 = make_float2(ex2(e2.x), ex2(e2.y)); e3 = make_float2(ex2(e3.x), ex2(e3.y));
+        a0 = __fadd2_rn(a0, e0); a1 = __fadd2_rn(a1, e1);
+        a2 = __fadd2_rn(a2, e2); a3 = __fadd2_rn(a3, e3);
+        pk[c / 2 + 0] = pack_bf16(e0.x, e0.y); pk[c / 2 + 1] = pack_bf16(e1.x, e1.y);
+        pk[c / 2 + 2] = pack_bf16(e2.x, e2.y); pk[c / 2 + 3] = pack_bf16(e3.x, e3.y);
+      }
+      a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+      l += a0.x + a0.y;
+      if (__any_sync(0xffffffffu, rescale)) {              // O_t *= corr (rare)
         uint32_t o0[32], o1[32];
-        tmem_ld32(tmem_o + lane_off, o0); tmem_ld32(tmem_o + lane_off + 32, o1);
+        tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           o0[c] = __float_as_uint(__uint_as_float(o0[c]) * corr);
           o1[c] = __float_as_uint(__uint_as_float(o1[c]) * corr);
         }
-        tmem_st32(tmem_o + lane_off, o0); tmem_st32(tmem_o + lane_off + 32, o1);
-        tmem_st_wait();
+        tmem_st32(tm_o, o0); tmem_st32(tm_o + 32, o1);
       }
-      float rowsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) { x[c] = ex2(x[c] - m_ref); rowsum += x[c]; }
-      l += rowsum;
-      // P buffer b was last read by the MMA of tile j-2
-      if (j >= 2 && !mbar_wait_warp(&p_free[b], ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-      uint8_t* prow = smem + S::kP + b * 32768 + r * 128;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const float* v = x + half * 64 + ch * 8;
-          uint4 u;
-          u.x = pack_bf16(v[0], v[1]); u.y = pack_bf16(v[2], v[3]);
-          u.z = pack_bf16(v[4], v[5]); u.w = pack_bf16(v[6], v[7]);
-          *reinterpret_cast<uint4*>(prow + half * 16384 + ((ch ^ (r & 7)) << 4)) = u;
-        }
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk + 32);
+        tmem_st32(tm_p, lo);
+        tmem_st32(tm_p + 32, hi);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait_warp(o_final, 0, abort_flag, p.status)) {
+    if (ok && mbar_wait_warp(&o_final[t], 0, abort_flag, p.status)) {
       tc_fence_after();
       uint32_t o0[32], o1[32];
-      tmem_ld32(tmem_o + lane_off, o0); tmem_ld32(tmem_o + lane_off + 32, o1);
+      tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
       tmem_ld_wait();
-      const int row = q0 + r;
+      const int row = q0 + t * 128 + r;
       if (row < p.L) {
         const float inv = 1.f / l;
         float v[64];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) { v[c] = __uint_as_float(o0[c]) * inv; v[32 + c] = __uint_as_float(o1[c]) * inv; }
+        for (int c = 0; c < 32; ++c) {
+          v[c] = __uint_as_float(o0[c]) * inv;
+          v[32 + c] = __uint_as_float(o1[c]) * inv;
+        }
         store_vec<bf16, 64>(static_cast<bf16*>(p.o) + size_t(row) * p.H * 64 + size_t(h) * 64, v);
       }
     }
