@@ -417,8 +417,9 @@ fd_status_t fd_handle::build_graph() {
       ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
       ap.fs = fs;
       ap.status = status;
-      // two query tiles per CTA when that still gives at least one full wave
-      const bool two = ((L + 255) / 256) * H >= num_sms;
+      // one 128-query tile per CTA, two CTAs per SM (measured faster than two
+      // query tiles sharing one CTA's K/V stages and MMA issuer)
+      const bool two = false;
       const void* f = two ? reinterpret_cast<const void*>(&tc_attn_kernel<2>)
                           : reinterpret_cast<const void*>(&tc_attn_kernel<1>);
       const int smem_bytes = two ? TcAttnSmem<2>::kAlloc : TcAttnSmem<1>::kAlloc;
@@ -650,10 +651,10 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
       const uint32_t box[3] = {64, 128, 1};
       FD_TRY(make_tmap(&h->tm_q, h->q, 3, dims, str, box));
     }
-    {   // K [NB*G][kv_rows][64]: box 64 x 128 x 1
+    {   // K [NB*G][kv_rows][64]: box 64 dims x 64 keys x 1
       const uint64_t dims[3] = {64, uint64_t(h->kv_rows), uint64_t(NB) * G};
       const uint64_t str[2] = {64 * 2, uint64_t(h->kv_rows) * 64 * 2};
-      const uint32_t box[3] = {64, 128, 1};
+      const uint32_t box[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_k, h->kc, 3, dims, str, box));
     }
     {   // V^T [NB*G][64][vt_pitch]: box 64 keys x 64 dims x 1

@@ -6,19 +6,23 @@
 // are always the contiguous range [0, n_valid*L) and softmax, being
 // invariant to the order of keys, needs no slot bookkeeping.
 //
-// One CTA = one head x QT query tiles of 128 (QT = 1 or 2), sharing every
-// K/V stage between the tiles. Warps:
-//   0            TMA: the Q tiles once, then per stage K (128 keys x 64) and
-//                the transposed V (64 x 128 keys, two 64-key halves)
+// One CTA = one head x QT query tiles of 128 (QT = 1 or 2). Keys are
+// consumed in tiles of 64; every K/V stage is shared by the QT query tiles.
+// Warps:
+//   0            TMA: the Q tiles once, then per stage K (64 keys x 64) and
+//                the transposed V (64 dims x 64 keys)
 //   1            TMEM allocator; lane 0 issues, per key tile j,
-//                S_t = Q_t K_j^T for every query tile t (SS form), then
-//                O_t += P_t V_{j-1} (TS form: P read from TMEM)
+//                S_t(j) = Q_t K_j^T (SS form) for every query tile t, then
+//                O_t += P_t(j-1) V_{j-1} (TS form: P read from TMEM)
 //   2 .. 1+4*QT  softmax, one warpgroup per query tile, one query row per
 //                thread: S row from TMEM, base-2 online softmax with lazy
 //                rescaling (O is rescaled in TMEM only when the running max
 //                grows by more than 2^8), P packed to bf16 into TMEM
-// TMEM columns: S_t [128 t, 128 t + 128), O_t [256 + 64 t, +64),
-//               P_t [384 + 64 t, +64) (128 bf16 keys packed 2 per column).
+// S and P are double-buffered per query tile, so the softmax of tile j runs
+// while the tensor core still computes S(j+1) and O += P(j-1) V(j-1); the
+// only waits on the critical path are for data two tiles old.
+// TMEM columns (64 fp32 S columns, 32 packed-bf16 P columns per buffer):
+//   S[t][b] at 64 (2t + b), O_t at 64 (2 QT + t), P[t][b] at 64 (3 QT) + 32 (2t + b).
 // Keys past n_valid*L inside the last tile get probability 0.
 #pragma once
 
@@ -37,16 +41,19 @@ struct TcAttnParams {
 
 template <int QT>
 struct TcAttnSmem {
-  static constexpr int kStages = QT == 2 ? 4 : 4;
+  static constexpr int kStages = QT == 2 ? 8 : 4;
   static constexpr int kQ = 0;                                // QT x 16 KB
-  static constexpr int kKV = QT * 16384;                      // stages x (K 16 KB + V 16 KB)
-  static constexpr int kKVStage = 32768;
+  static constexpr int kKV = QT * 16384;                      // stages x (K 8 KB + V^T 8 KB)
+  static constexpr int kKVStage = 16384;
   static constexpr int kBar = kKV + kStages * kKVStage;
-  // q_full, kv_full[ST], kv_empty[ST], s_full[2], s_free[2], p_full[2], p_free[2], o_final[2]
-  static constexpr int kNumBars = 1 + 2 * kStages + 10;
+  // q_full, kv_full[ST], kv_empty[ST], then per tile: s_full[2], s_free[2],
+  // p_full[2], p_free[2], o_final
+  static constexpr int kNumBars = 1 + 2 * kStages + 9 * QT;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr int kThreads = 64 + 128 * QT;
+  static constexpr int kTmemCols = QT == 2 ? 512 : 256;
+  static constexpr int kMinBlocks = QT == 2 ? 1 : 2;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -92,15 +99,37 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// p = 2^(s * sc - m) for one 64-key S row: packed bf16 pairs into pk[32];
+// returns the row sum. Scores of masked keys are -inf and give exactly 0.
+__device__ __forceinline__ float exp_pack64(const float* x, float sc, float m, uint32_t* pk) {
+  const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
+  float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+  for (int c = 0; c < 64; c += 8) {
+    float2 e0 = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nm2);
+    float2 e1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), sc2, nm2);
+    float2 e2 = __ffma2_rn(make_float2(x[c + 4], x[c + 5]), sc2, nm2);
+    float2 e3 = __ffma2_rn(make_float2(x[c + 6], x[c + 7]), sc2, nm2);
+    e0 = make_float2(ex2(e0.x), ex2(e0.y)); e1 = make_float2(ex2(e1.x), ex2(e1.y));
+    e2 = make_float2(ex2(e2.x), ex2(e2.y)); e3 = make_float2(ex2(e3.x), ex2(e3.y));
+    a0 = __fadd2_rn(a0, e0); a1 = __fadd2_rn(a1, e1);
+    a2 = __fadd2_rn(a2, e2); a3 = __fadd2_rn(a3, e3);
+    pk[c / 2 + 0] = pack_bf16(e0.x, e0.y); pk[c / 2 + 1] = pack_bf16(e1.x, e1.y);
+    pk[c / 2 + 2] = pack_bf16(e2.x, e2.y); pk[c / 2 + 3] = pack_bf16(e3.x, e3.y);
+  }
+  a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+  return a0.x + a0.y;
+}
+
 template <int QT>
-__global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
+__global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMinBlocks)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcAttnParams p) {
   using S = TcAttnSmem<QT>;
   constexpr int ST = S::kStages;
-  constexpr uint32_t kTmemCols = 512;
-  constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128);
-  constexpr uint32_t kIdescO = idesc_bf16_f32(128, 64);
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64);   // 128 queries x 64 keys
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, 64);   // 128 queries x 64 dims
+  constexpr uint32_t kColO = 64 * 2 * QT, kColP = 64 * 3 * QT;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -109,34 +138,37 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + ST;
-  uint64_t* s_full = kv_empty + ST;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* p_free = p_full + 2;
-  uint64_t* o_final = p_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 2);
+  uint64_t* tb = kv_empty + ST;                 // per tile t: 9 barriers at tb + 9 t
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tb + 9 * QT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto s_full = [&](int t, int b) { return tb + 9 * t + b; };
+  auto s_free = [&](int t, int b) { return tb + 9 * t + 2 + b; };
+  auto p_full = [&](int t, int b) { return tb + 9 * t + 4 + b; };
+  auto p_free = [&](int t, int b) { return tb + 9 * t + 6 + b; };
+  auto o_final = [&](int t) { return tb + 9 * t + 8; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = blockIdx.x * (128 * QT), h = blockIdx.y;
   const int g = h / (p.H / p.G);
   const int lg = p.layer * p.G + g;
   const int n_keys = p.fs->n_valid * p.L;
-  const int n_kt = (n_keys + 127) / 128;
+  const int n_kt = (n_keys + 63) / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1); mbar_init(&s_free[t], 128);
-      mbar_init(&p_full[t], 128); mbar_init(&p_free[t], 1);
-      mbar_init(&o_final[t], 1);
+    for (int t = 0; t < QT; ++t) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(s_full(t, b), 1); mbar_init(s_free(t, b), 128);
+        mbar_init(p_full(t, b), 128); mbar_init(p_free(t, b), 1);
+      }
+      mbar_init(o_final(t), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmQ); prefetch_tensormap(&tmK); prefetch_tensormap(&tmV);
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, kTmemCols); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(tmem_slot, S::kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -152,127 +184,104 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
         if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* kv = smem + S::kKV + st * S::kKVStage;
         mbar_arrive_expect_tx(&kv_full[st], S::kKVStage);
-        tma_load_3d(kv, &tmK, 0, j * 128, lg, &kv_full[st]);
-        tma_load_3d(kv + 16384, &tmV, j * 128, 0, lg, &kv_full[st]);
-        tma_load_3d(kv + 16384 + 8192, &tmV, j * 128 + 64, 0, lg, &kv_full[st]);
+        tma_load_3d(kv, &tmK, 0, j * 64, lg, &kv_full[st]);
+        tma_load_3d(kv + 8192, &tmV, j * 64, 0, lg, &kv_full[st]);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {                                       // ---- MMA issuer
-      // O_t += P_t(i) V(i): A from TMEM (P_t), B = V^T halves in shared memory
-      auto issue_pv = [&](int t, int i) -> bool {
-        if (!mbar_wait(&p_full[t], i & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(smem + S::kKV + (i % ST) * S::kKVStage + 16384);
-        const uint32_t a_tm = tmem_base + 384 + 64 * t;
-        const uint32_t d_tm = tmem_base + 256 + 64 * t;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_ts(d_tm, a_tm + 8 * k, sw128_desc(sv + (k >> 2) * 8192) + 2 * (k & 3), kIdescO,
-                    (i | k) != 0);
-        tc_commit(&p_free[t]);
-        return true;
-      };
+    // Two MMA issuers, so S(j+1) never waits behind O += P(j-1) V(j-1):
+    // lane 0 issues S_t(j) = Q_t K_j^T as soon as an S buffer is free;
+    // lane 1 issues O_t += P_t(j) V_j as soon as P_t(j) is written, then
+    // releases the K/V stage (S(j) precedes P(j), so K is no longer read).
+    // Each lane's tcgen05.commit tracks only its own MMAs.
+    if (lane == 0) {                                       // ---- S issuer
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < n_kt; ++j) {
-        const int st = j % ST;
-        if (!mbar_wait(&kv_full[st], (j / ST) & 1, abort_flag, p.status)) { ok = false; break; }
+        const int st = j % ST, b = j & 1;
+        if (!mbar_wait(&kv_full[st], (j / ST) & 1, abort_flag, p.status)) break;
         const uint32_t sk = smem_u32(smem + S::kKV + st * S::kKVStage);
         for (int t = 0; t < QT; ++t) {
-          if (!mbar_wait(&s_free[t], (j & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait(s_free(t, b), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sq = smem_u32(smem + S::kQ + t * 16384);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_ss(tmem_base + 128 * t, sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k, kIdescS,
-                      k != 0);
-          tc_commit(&s_full[t]);
-        }
-        if (!ok) break;
-        if (j >= 1) {
-          for (int t = 0; t < QT && ok; ++t) ok = issue_pv(t, j - 1);
-          if (ok) tc_commit(&kv_empty[(j - 1) % ST]);
+            tc_mma_ss(tmem_base + 64 * (2 * t + b), sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k,
+                      kIdescS, k != 0);
+          tc_commit(s_full(t, b));
         }
       }
-      if (ok) {
-        for (int t = 0; t < QT && ok; ++t) ok = issue_pv(t, n_kt - 1);
-        if (ok)
-          for (int t = 0; t < QT; ++t) tc_commit(&o_final[t]);
+    } else if (lane == 1) {                                // ---- PV issuer
+      bool ok = true;
+      for (int i = 0; ok && i < n_kt; ++i) {
+        const int b = i & 1;
+        const uint32_t sv = smem_u32(smem + S::kKV + (i % ST) * S::kKVStage + 8192);
+        for (int t = 0; t < QT; ++t) {
+          if (!mbar_wait(p_full(t, b), (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_tm = tmem_base + kColP + 32 * (2 * t + b);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_ts(tmem_base + kColO + 64 * t, a_tm + 8 * k, sw128_desc(sv) + 2 * k, kIdescO,
+                      (i | k) != 0);
+          tc_commit(p_free(t, b));
+        }
+        if (ok) tc_commit(&kv_empty[i % ST]);
       }
+      if (ok)
+        for (int t = 0; t < QT; ++t) tc_commit(o_final(t));
     }
   } else {                                                 // ---- softmax warpgroups
     const int t = (warp - 2) >> 2;                         // query tile of this warpgroup
     const int quarter = warp & 3;                          // TMEM lanes 32*quarter ..
     const int r = quarter * 32 + lane;                     // query row within the tile
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t tm_s = tmem_base + lane_off + 128 * t;
-    const uint32_t tm_o = tmem_base + lane_off + 256 + 64 * t;
-    const uint32_t tm_p = tmem_base + lane_off + 384 + 64 * t;
+    const uint32_t tm_o = tmem_base + lane_off + kColO + 64 * t;
     const float sc = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
-      if (!mbar_wait_warp(&s_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
+      const int b = j & 1;
+      if (!mbar_wait_warp(s_full(t, b), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
+      float x[64];
       {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tm_s, r0); tmem_ld32(tm_s + 32, r1); tmem_ld32(tm_s + 64, r2);
-        tmem_ld32(tm_s + 96, r3);
+        uint32_t r0[32], r1[32];
+        const uint32_t tm_s = tmem_base + lane_off + 64 * (2 * t + b);
+        tmem_ld32(tm_s, r0); tmem_ld32(tm_s + 32, r1);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]);
-          x[64 + c] = __uint_as_float(r2[c]); x[96 + c] = __uint_as_float(r3[c]);
-        }
+        for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
       }
       tc_fence_before();
-      mbar_arrive(&s_free[t]);
-      const int valid = n_keys - j * 128;                  // keys of this tile in range
-      if (valid < 128) {
+      mbar_arrive(s_free(t, b));
+      const int valid = n_keys - j * 64;                   // keys of this tile in range
+      if (valid < 64) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
+        for (int c = 0; c < 64; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
       }
       // row max of the raw scores (the scale is positive)
       float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
-      float m2 = max3(x[6], x[7], x[8]), m3 = max3(x[9], x[10], x[11]);
 #pragma unroll
-      for (int c = 12; c < 124; c += 8) {
-        m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]);
-        m2 = max3(m2, x[c + 4], x[c + 5]); m3 = max3(m3, x[c + 6], x[c + 7]);
-      }
-      m0 = max3(m0, x[124], x[125]); m1 = max3(m1, x[126], x[127]);
-      const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sc;
+      for (int c = 6; c < 62; c += 4) { m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]); }
+      m0 = max3(m0, x[62], x[63]);
+      const float mx = fmaxf(m0, m1) * sc;
       bool rescale = false;
       if (j == 0) m_ref = mx;
       else if (mx > m_ref + 8.f) rescale = true;
-      // P_t and O_t are free once the MMA of the previous tile has finished
-      if (j >= 1) {
-        if (!mbar_wait_warp(&p_free[t], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-      }
       const float corr = rescale ? ex2(m_ref - mx) : 1.f;
       if (rescale) { m_ref = mx; l *= corr; }
-      // p = 2^(s * scale - m_ref), packed fp32 pairs; row sum in 4 partials
-      const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m_ref, -m_ref);
-      float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        float2 e0 = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nm2);
-        float2 e1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), sc2, nm2);
-        float2 e2 = __ffma2_rn(make_float2(x[c + 4], x[c + 5]), sc2, nm2);
-        float2 e3 = __ffma2_rn(make_float2(x[c + 6], x[c + 7]), sc2, nm2);
-        e0 = make_float2(ex2(e0.x), ex2(e0.y)); e1 = make_float2(ex2(e1.x), ex2(e1.y));
-        e2 = make_float2(ex2(e2.x), ex2(e2.y)); e3 = make_float2(ex2(e3.x), ex2(e3.y));
-        a0 = __fadd2_rn(a0, e0); a1 = __fadd2_rn(a1, e1);
-        a2 = __fadd2_rn(a2, e2); a3 = __fadd2_rn(a3, e3);
-        pk[c / 2 + 0] = pack_bf16(e0.x, e0.y); pk[c / 2 + 1] = pack_bf16(e1.x, e1.y);
-        pk[c / 2 + 2] = pack_bf16(e2.x, e2.y); pk[c / 2 + 3] = pack_bf16(e3.x, e3.y);
+      uint32_t pk[32];
+      l += exp_pack64(x, sc, m_ref, pk);
+      // P buffer b was last read by the MMA of tile j-2
+      if (j >= 2) {
+        if (!mbar_wait_warp(p_free(t, b), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
       }
-      a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
-      l += a0.x + a0.y;
-      if (__any_sync(0xffffffffu, rescale)) {              // O_t *= corr (rare)
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_t *= corr (rare): every earlier O += P V must have landed first
+        if (!mbar_wait_warp(p_free(t, b ^ 1), ((j - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
         uint32_t o0[32], o1[32];
         tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
         tmem_ld_wait();
@@ -283,17 +292,12 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
         }
         tmem_st32(tm_o, o0); tmem_st32(tm_o + 32, o1);
       }
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk + 32);
-        tmem_st32(tm_p, lo);
-        tmem_st32(tm_p + 32, hi);
-      }
+      tmem_st32(tmem_base + lane_off + kColP + 32 * (2 * t + b), pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(p_full(t, b));
     }
-    if (ok && mbar_wait_warp(&o_final[t], 0, abort_flag, p.status)) {
+    if (ok && mbar_wait_warp(o_final(t), 0, abort_flag, p.status)) {
       tc_fence_after();
       uint32_t o0[32], o1[32];
       tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, S::kTmemCols);
   }
 }
 

@@ -7,7 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/flashdec.h"
+#include "flashdec.h"
 
 namespace fd {
 
