@@ -142,22 +142,27 @@ def barrier(dist):
         dist.barrier()
 
 
-def max_over_ranks(dist, v):
-    if dist is None:
-        return v
+def _reduce(dist, v, op):
     import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(dist, v):
+    """Timing of a replicated step: the slowest rank's time."""
+    return v if dist is None else _reduce(dist, v, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(dist, v):
-    if dist is None:
-        return v
-    import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    """Work of a replicated step: the units all ranks processed."""
+    return v if dist is None else _reduce(dist, v, dist.ReduceOp.SUM)
+
+
+def replica_throughput(r_t, frames_all_ranks, max_ms):
+    """Whole-job pixel frames per second of N independent decoders."""
+    return r_t * frames_all_ranks / (max_ms / 1e3)
 
 
 # ------------------------------------------------------------------ oracle
@@ -284,7 +289,7 @@ def run_flashdec(args):
     total_ms = max_over_ranks(dist, total_ms)
     lat_ms = [a.elapsed_time(b) for a, b in ev]
     frames_all = sum_over_ranks(dist, args.steps)
-    value = cfg.r_t * frames_all / (total_ms / 1e3)
+    value = replica_throughput(cfg.r_t, frames_all, total_ms)
     kernels_per_frame = len(dec.kernel_ms())
 
     # ---- end to end: host buffers through fd_decode_frame_host

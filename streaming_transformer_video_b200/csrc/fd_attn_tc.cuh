@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
         const uint32_t tm_s = tmem_base + lane_off + 64 * (2 * t + b);
         tmem_ld32(tm_s, r0); tmem_ld32(tm_s + 32, r1);
         tmem_ld_wait();
+        reg_fence(r0); reg_fence(r1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
       }
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
         uint32_t o0[32], o1[32];
         tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
         tmem_ld_wait();
+        reg_fence(o0); reg_fence(o1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           o0[c] = __float_as_uint(__uint_as_float(o0[c]) * corr);
@@ -302,6 +304,7 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
       uint32_t o0[32], o1[32];
       tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
       tmem_ld_wait();
+      reg_fence(o0); reg_fence(o1);
       const int row = q0 + t * 128 + r;
       if (row < p.L) {
         const float inv = 1.f / l;

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld32(taddr + c, r0);
         tmem_ld32(taddr + c + 32, r1);
         tmem_ld_wait();
+        reg_fence(r0);
+        reg_fence(r1);
         float acc[64];
 #pragma unroll
         for (int i = 0; i < 32; ++i) { acc[i] = __uint_as_float(r0[i]); acc[32 + i] = __uint_as_float(r1[i]); }

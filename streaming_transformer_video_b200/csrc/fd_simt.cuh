@@ -48,7 +48,7 @@ struct EmbedParams {
   float* ssq;             // [L][D/32]
 };
 
-constexpr int kEmbedTok = 8;
+constexpr int kEmbedTok = 32;
 
 // One CTA = kEmbedTok tokens; thread d handles columns d, d+256, ...
 // Sums of squares per 32-column chunk come from a warp reduction (each warp
