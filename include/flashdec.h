@@ -74,8 +74,10 @@ typedef struct {
   fd_dtype io_dtype;     /* element type of latent_frame and out_pixels           */
   float norm_eps;        /* RMSNorm epsilon (1e-6)                                */
   float rope_theta;      /* RoPE base (1e4)                                       */
-  int32_t kernel_timing; /* 1: bracket each kernel with CUDA events (for
-                            fd_last_step_kernel_ms); 0: off                       */
+  int32_t kernel_timing; /* CUDA events recorded inside the graph, read by
+                            fd_last_step_kernel_ms: 0 off; 1 around every
+                            kernel; 2 around each attention launch only (the
+                            dominant kernel; negligible overhead)                */
 } fd_config;
 
 /*
@@ -178,11 +180,12 @@ FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
 
 /*
- * Kernel timing (requires cfg.kernel_timing = 1): waits for the last
- * enqueued frame and writes the device time in ms of each kernel of that
- * frame, in launch order, to ms_out[0 .. n-1] and its kernel kind to
- * kind_out (see fd_kernel_kind). *n_out = number of kernels in one frame.
- * Pass cap = 0 to query *n_out only.
+ * Kernel timing (requires cfg.kernel_timing = 1 or 2): waits for the last
+ * enqueued frame and writes the device time in ms of each timed kernel of
+ * that frame (every kernel, or every attention launch), in launch order, to
+ * ms_out[0 .. n-1] and its kind to kind_out (see fd_kernel_kind).
+ * *n_out = number of timed kernels per frame. Pass cap = 0 to query *n_out
+ * only. Each replay of the frame graph overwrites the previous frame's times.
  */
 typedef enum {
   FD_K_STEP_BEGIN = 0, FD_K_EMBED = 1, FD_K_QKV = 2, FD_K_ATTN = 3,
@@ -190,6 +193,18 @@ typedef enum {
 } fd_kernel_kind;
 FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out,
                                    int32_t cap, int32_t* n_out);
+
+/*
+ * Self-test of the device-side failure path (no handle needed; runs on the
+ * current device and synchronises it). Every device wait of the decoder's
+ * kernels is bounded; this launches one tiny kernel that waits, with the same
+ * bounded-wait code and a limit of timeout_us microseconds (1 .. 10^7), on an
+ * mbarrier that nothing ever completes. Returns FD_ERR_TIMEOUT when the wait
+ * gave up as designed and the GPU context is still usable afterwards, FD_OK
+ * if the wait wrongly succeeded, FD_ERR_INVALID_ARG for a bad limit and
+ * FD_ERR_CUDA for a runtime failure. No fault, trap or hang is involved.
+ */
+FD_API fd_status_t fd_selftest_wait_timeout(int32_t timeout_us);
 
 #ifdef __cplusplus
 }

@@ -166,7 +166,9 @@ struct fd_handle {
   const void* cur_latent = nullptr;
   void* cur_out = nullptr;
   std::vector<cudaEvent_t> events;
-  std::vector<int> kinds;
+  std::vector<int> kinds;               // fd_kernel_kind of every kernel node, in order
+  struct Timed { int begin, end, kind; };
+  std::vector<Timed> timed;             // kernels bracketed by event pairs
   cudaStream_t last_stream = nullptr;
 
   // ---------------------------------------------------------------- memory
@@ -230,7 +232,15 @@ struct fd_handle {
     last_node = n;
     return FD_OK;
   }
+  // kernel_timing 1: one event after every kernel (consecutive events bracket
+  // each kernel); 2: an event pair around each attention launch only.
   fd_status_t add_kernel(const KernelLaunch& k, void** args, cudaGraphNode_t* out_node = nullptr) {
+    const bool bracket = cfg.kernel_timing == 2 && k.kind == FD_K_ATTN;
+    int begin = int(events.size()) - 1;
+    if (bracket) {
+      FD_TRY(add_event());
+      begin = int(events.size()) - 1;
+    }
     cudaKernelNodeParams np{};
     np.func = const_cast<void*>(k.func);
     np.gridDim = k.grid;
@@ -243,7 +253,10 @@ struct fd_handle {
     last_node = n;
     if (out_node) *out_node = n;
     kinds.push_back(k.kind);
-    if (cfg.kernel_timing) FD_TRY(add_event());
+    if (cfg.kernel_timing == 1 || bracket) {
+      FD_TRY(add_event());
+      timed.push_back({begin, int(events.size()) - 1, k.kind});
+    }
     return FD_OK;
   }
 
@@ -267,7 +280,7 @@ fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   const int tiles = ((M + 127) / 128) * (N / BN);
   k->func = f;
   k->grid = dim3(std::min(tiles, num_sms));
-  k->block = dim3(192);
+  k->block = dim3(kGemmThreads);
   k->smem = S::kAlloc;
   return FD_OK;
 }
@@ -358,7 +371,7 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
 fd_status_t fd_handle::build_graph() {
   FD_CUDA(cudaGraphCreate(&graph, 0));
   last_node = nullptr;
-  if (cfg.kernel_timing) FD_TRY(add_event());
+  if (cfg.kernel_timing == 1) FD_TRY(add_event());
 
   // step_begin
   {
@@ -418,15 +431,11 @@ fd_status_t fd_handle::build_graph() {
       ap.fs = fs;
       ap.status = status;
       // one 128-query tile per CTA, two CTAs per SM (measured faster than two
-      // query tiles sharing one CTA's K/V stages and MMA issuer)
-      const bool two = false;
-      const void* f = two ? reinterpret_cast<const void*>(&tc_attn_kernel<2>)
-                          : reinterpret_cast<const void*>(&tc_attn_kernel<1>);
-      const int smem_bytes = two ? TcAttnSmem<2>::kAlloc : TcAttnSmem<1>::kAlloc;
-      const int threads = two ? TcAttnSmem<2>::kThreads : TcAttnSmem<1>::kThreads;
-      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes));
-      const int qrows = two ? 256 : 128;
-      KernelLaunch k{f, dim3((L + qrows - 1) / qrows, H), dim3(threads), size_t(smem_bytes),
+      // query tiles sharing one CTA, and than three CTAs with single-buffered S)
+      using A = TcAttnSmem<1>;
+      const void* f = reinterpret_cast<const void*>(&tc_attn_kernel<1>);
+      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
+      KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(A::kThreads), size_t(A::kAlloc),
                      FD_K_ATTN};
       CUtensorMap a = tm_q, b = tm_k, c = tm_v;
       void* args[] = {&a, &b, &c, &ap};
@@ -530,8 +539,8 @@ fd_status_t validate(const fd_config* c) {
   if (L * (c->window + 1) > (1LL << 30))
     return fail(FD_ERR_UNSUPPORTED, "config: window of %lld tokens is too large",
                 L * (c->window + 1));
-  if (c->kernel_timing != 0 && c->kernel_timing != 1)
-    return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0 or 1");
+  if (c->kernel_timing < 0 || c->kernel_timing > 2)
+    return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0, 1 or 2");
   return FD_OK;
 }
 
@@ -888,11 +897,39 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
   return FD_OK;
 }
 
+fd_status_t fd_selftest_wait_timeout(int32_t timeout_us) {
+  g_last_error.clear();
+  if (timeout_us < 1 || timeout_us > 10000000)
+    return fail(FD_ERR_INVALID_ARG, "fd_selftest_wait_timeout: limit out of range");
+  int* d_status = nullptr;
+  FD_CUDA(cudaMalloc(&d_status, 4));
+  fd_status_t result = FD_OK;
+  int st = 0;
+  cudaError_t e = cudaMemset(d_status, 0, 4);
+  if (e == cudaSuccess) {
+    wait_timeout_selftest_kernel<<<1, 32>>>(d_status, 1000ull * timeout_us);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&st, d_status, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(d_status, 0, 4);     // the context still works
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(d_status);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FD_ERR_CUDA, "fd_selftest_wait_timeout: %s", cudaGetErrorString(e));
+  }
+  result = fd_status_t(st);
+  if (result == FD_ERR_TIMEOUT) fail(FD_ERR_TIMEOUT, "device wait gave up after %d us as designed",
+                                     timeout_us);
+  return result;
+}
+
 fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out, int32_t cap,
                                    int32_t* n_out) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_last_step_kernel_ms: invalid handle");
   if (!n_out) return fail(FD_ERR_INVALID_ARG, "fd_last_step_kernel_ms: null n_out");
-  const int n = int(h->kinds.size());
+  const int n = int(h->timed.size());
   *n_out = n;
   if (cap == 0) return FD_OK;
   if (!h->cfg.kernel_timing)
@@ -902,9 +939,9 @@ fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_ou
   FD_CUDA(cudaEventSynchronize(h->events.back()));
   for (int i = 0; i < n; ++i) {
     float ms = 0.f;
-    FD_CUDA(cudaEventElapsedTime(&ms, h->events[i], h->events[i + 1]));
+    FD_CUDA(cudaEventElapsedTime(&ms, h->events[h->timed[i].begin], h->events[h->timed[i].end]));
     ms_out[i] = ms;
-    kind_out[i] = h->kinds[i];
+    kind_out[i] = h->timed[i].kind;
   }
   return FD_OK;
 }

@@ -10,6 +10,7 @@
 //               K=16 per instruction, 4 per 64-wide stage) and commits
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, one
 //               token row per thread, fused epilogue (fd_epilogue.cuh)
+//               (eight epilogue warps, two per row group, measured no faster)
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the
 // epilogue of tile i overlaps the main loop of tile i+1. Tiles are handed out
 // round-robin over a grid of at most one CTA per SM. Rows past M are read as
@@ -32,8 +33,11 @@ struct TcGemmSmem {
   static constexpr int kAlloc = kBytes + 1024;        // slack for 1024-B alignment
 };
 
+constexpr int kEpiThreads = 128;                       // 4 epilogue warps
+constexpr int kGemmThreads = 64 + kEpiThreads;
+
 template <int BN, int STAGES, int KIND, int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int K, EpiParams ep, int* status) {
   using S = TcGemmSmem<BN, STAGES>;
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], kEpiThreads); }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
@@ -113,8 +117,11 @@ __global__ void __launch_bounds__(192, 1)
         tc_commit(&acc_full[buf]);          // accumulator ready for the epilogue
       }
     }
-  } else {                                            // ---- epilogue warps 2..5
+  } else {                                            // ---- epilogue warps
+    // kEpiThreads / 128 warps per TMEM lane quarter, alternate 64-column chunks
+    constexpr int kPerQuarter = kEpiThreads / 128;
     const int quarter = warp & 3;                     // TMEM lanes 32*quarter ..
+    const int half = (warp - 2) >> 2;
     int it = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int m_blk = tile / n_n, n_blk = tile - (tile / n_n) * n_n;
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(192, 1)
       if (KIND != EPI_RESID && row < M) rs = row_scale(ep, row);
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + buf * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 64) {
+      for (int c = 64 * half; c < BN; c += 64 * kPerQuarter) {
         uint32_t r0[32], r1[32];
         tmem_ld32(taddr + c, r0);
         tmem_ld32(taddr + c + 32, r1);

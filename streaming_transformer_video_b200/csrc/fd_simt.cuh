@@ -9,6 +9,7 @@
 #pragma once
 
 #include "fd_epilogue.cuh"
+#include "fd_ptx.cuh"
 
 namespace fd {
 
@@ -33,6 +34,22 @@ __global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int hea
   *ctr = t + 1;
 }
 
+// ---------------------------------------------------------------- self-test
+// Exercises the bounded-wait path every tcgen05 kernel relies on: an mbarrier
+// that nobody arrives on is waited for with the same helper and a short
+// limit; the wait must give up and record FD_ERR_TIMEOUT in *status.
+__global__ void wait_timeout_selftest_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, timeout_ns);
+}
+
 // ---------------------------------------------------------------- embed
 struct EmbedParams {
   const void* latent;     // [C'][H'][W'] io type
@@ -48,7 +65,7 @@ struct EmbedParams {
   float* ssq;             // [L][D/32]
 };
 
-constexpr int kEmbedTok = 32;
+constexpr int kEmbedTok = 8;
 
 // One CTA = kEmbedTok tokens; thread d handles columns d, d+256, ...
 // Sums of squares per 32-column chunk come from a warp reduction (each warp

@@ -24,7 +24,8 @@ KERNEL_KINDS = ["step_begin", "embed", "qkv", "attn", "oproj", "mlp_up", "mlp_do
 
 EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
-           "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms"]
+           "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
+           "fd_selftest_wait_timeout"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -73,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_debug_read_slot.argtypes = [vp, i32, i32, i32, _PF]
     lib.fd_last_step_kernel_ms.argtypes = [vp, _PF, ctypes.POINTER(i32), i32,
                                            ctypes.POINTER(i32)]
+    lib.fd_selftest_wait_timeout.argtypes = [i32]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
             getattr(lib, name).restype = i32
@@ -110,6 +112,12 @@ def _dtype_code(s) -> int:
     raise ValueError(f"unknown dtype {s!r}")
 
 
+def selftest_wait_timeout(timeout_us: int) -> int:
+    """Run the device-side bounded-wait self-test; returns the fd status code
+    (FD_ERR_TIMEOUT when the wait gave up as designed)."""
+    return int(lib().fd_selftest_wait_timeout(int(timeout_us)))
+
+
 def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
     """fd_config from any object with the decoder's shape attributes."""
     c = FDConfigC()
@@ -121,7 +129,8 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
     c.io_dtype = _dtype_code(io_dtype if io_dtype is not None else cfg.dtype)
     c.norm_eps = float(getattr(cfg, "norm_eps", 1e-6))
     c.rope_theta = float(getattr(cfg, "rope_theta", 1e4))
-    c.kernel_timing = 1 if kernel_timing else 0
+    # False/0: off; True/1: every kernel; 2: attention launches only
+    c.kernel_timing = int(kernel_timing)
     return c
 
 
@@ -236,7 +245,7 @@ class FlashDecoder:
         return out
 
     def kernel_ms(self) -> List[Tuple[str, float]]:
-        """(kind, ms) of every kernel of the last frame (kernel_timing=True)."""
+        """(kind, ms) of every timed kernel of the last frame (kernel_timing 1 or 2)."""
         n = ctypes.c_int32()
         _check(self._lib.fd_last_step_kernel_ms(self.h, None, None, 0, ctypes.byref(n)),
                "fd_last_step_kernel_ms")

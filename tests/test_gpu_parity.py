@@ -231,3 +231,27 @@ def test_480p_full_size_frames_0_to_3_match_oracle():
     got = gpu_decode(cfg, w, z)
     ref = oracle_decode(cfg, w, z)
     assert_close(cfg, got, ref)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_kernel_timing_modes(mode):
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder
+    cfg = small_bf16(frames=3)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    dec = FlashDecoder(cfg, w, kernel_timing=mode)
+    dec.reset()
+    lat = torch.from_numpy(z).to(torch.bfloat16).cuda()
+    out = torch.empty(cfg.out_shape, dtype=torch.bfloat16, device="cuda")
+    for t in range(3):
+        dec.decode_frame(lat[t], out)
+    times = dec.kernel_ms()
+    dec.close()
+    kinds = [k for k, _ in times]
+    if mode == 1:                       # every kernel of the frame, in launch order
+        assert kinds == ["step_begin", "embed"] + \
+            ["qkv", "attn", "oproj", "mlp_up", "mlp_down"] * cfg.n_blocks + ["final"]
+    else:                               # the attention launches only
+        assert kinds == ["attn"] * cfg.n_blocks
+    assert all(ms > 0 for _, ms in times)
