@@ -61,10 +61,19 @@ struct EpiParams {
 };
 
 __device__ __forceinline__ float row_scale(const EpiParams& p, int row) {
-  const float* s = p.ssq + size_t(row) * p.ssq_parts;
-  float acc = 0.f;
-  for (int i = 0; i < p.ssq_parts; ++i) acc += s[i];
-  return rsqrtf(acc * p.inv_d + p.eps);
+  // ssq_parts = D / 32 is even (D is a multiple of 64): independent loads in
+  // flight, four partial sums
+  const float2* s = reinterpret_cast<const float2*>(p.ssq + size_t(row) * p.ssq_parts);
+  const int n2 = p.ssq_parts / 2;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int i = 0;
+#pragma unroll 4
+  for (; i + 2 <= n2; i += 2) {
+    const float2 u = s[i], v = s[i + 1];
+    a0 += u.x; a1 += u.y; a2 += v.x; a3 += v.y;
+  }
+  if (i < n2) { const float2 u = s[i]; a0 += u.x; a1 += u.y; }
+  return rsqrtf(((a0 + a1) + (a2 + a3)) * p.inv_d + p.eps);
 }
 
 __device__ __forceinline__ float gelu_erf(float x) {
