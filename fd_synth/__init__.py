@@ -111,6 +111,11 @@ CONFIGS: Dict[str, FDConfig] = {
     # 200 frames, 16 blocks.
     "long720p_wan22": FDConfig("long720p_wan22", 48, 45, 80, 1, 1024, 16, 16,
                                64, 16, 4, 2, 3, 4, 16, 1, "bf16", 200),
+    # FlashDecoder-XL backbone shape (D=1536, 24 heads, 3 KV groups, 20 blocks;
+    # the paper's W_frm=2 window = 1 past frame) on the Wan2.2 480p latent
+    # (48ch, 30x52 grid, 1560 tokens), 7 latent frames.
+    "xl_480p_wan22": FDConfig("xl_480p_wan22", 48, 30, 52, 1, 1536, 24, 3, 64,
+                              20, 4, 1, 3, 4, 16, 1, "bf16", 7),
 }
 
 

@@ -202,6 +202,9 @@ def test_nan_latent_propagates_without_failure():
     dict(window=3, frames=6),
     dict(grid_h=17, grid_w=23, frames=4),            # 391 tokens: 4 tiles, ragged
     dict(px_per_token=8),
+    dict(n_heads=8, n_kv_heads=1, d_model=512),      # GQA, 8 query heads per group
+    # FlashDecoder-XL block shape: D=1536, 24 heads, 3 KV groups (GQA ratio 8)
+    dict(d_model=1536, n_heads=24, n_kv_heads=3, n_blocks=1, window=1, frames=4),
 ])
 def test_small_bf16_matches_oracle(kw):
     cfg = small_bf16(**kw)
@@ -255,3 +258,14 @@ def test_kernel_timing_modes(mode):
     else:                               # the attention launches only
         assert kinds == ["attn"] * cfg.n_blocks
     assert all(ms > 0 for _, ms in times)
+
+
+def test_xl_gqa_480p_full_depth_frames_0_to_2_match_oracle():
+    # the FlashDecoder-XL backbone shape (D=1536, 24 query heads sharing 3
+    # key/value groups, 20 blocks, one past frame) on the 480p Wan2.2 latent
+    cfg = fd_synth.CONFIGS["xl_480p_wan22"]
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg, frames=3)
+    got = gpu_decode(cfg, w, z)
+    ref = oracle_decode(cfg, w, z)
+    assert_close(cfg, got, ref)
