@@ -53,6 +53,13 @@ class FDConfig:
     frames: int           # T' of the workload
     norm_eps: float = 1e-6
     rope_theta: float = 10000.0
+    # output head: "linear" = final RMSNorm + one Linear D -> C r_t P^2 +
+    # unpatchify; "paper" = temporal upsample Linear D -> r_t D (Eq. 3),
+    # n_refine streaming refinement blocks over the r_t sub-frames (window of
+    # r_t (W+1) sub-frames), RMSNorm + 2-layer MLP D -> D -> C P^2 and
+    # PixelShuffle per sub-frame (paper Sec. 3.4)
+    head: str = "linear"
+    n_refine: int = 2
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property
@@ -82,6 +89,11 @@ class FDConfig:
     @property
     def c_out(self) -> int:
         return self.out_ch * self.r_t * self.px_per_token * self.px_per_token
+
+    @property
+    def c_px(self) -> int:
+        """Columns of one sub-frame's spatial MLP output: C P^2."""
+        return self.out_ch * self.px_per_token * self.px_per_token
 
     @property
     def out_shape(self):
@@ -119,14 +131,23 @@ CONFIGS: Dict[str, FDConfig] = {
 }
 
 
+BLOCK_KEYS = ("norm1_g", "wqkv", "bqkv", "knorm_g", "vnorm_g", "wo", "bo", "norm2_g",
+              "w1", "b1", "w2", "b2")
+
+
 def weight_names(cfg: FDConfig) -> List[str]:
-    """Flat list of weight tensor names in generation order."""
+    """Flat list of weight tensor names in generation order. Backbone blocks
+    are "b{l}.*"; with the paper head, refinement blocks are "r{l}.*"."""
     names = ["embed_w", "embed_b"]
     for l in range(cfg.n_blocks):
-        names += [f"b{l}.norm1_g", f"b{l}.wqkv", f"b{l}.bqkv", f"b{l}.knorm_g",
-                  f"b{l}.vnorm_g", f"b{l}.wo", f"b{l}.bo", f"b{l}.norm2_g",
-                  f"b{l}.w1", f"b{l}.b1", f"b{l}.w2", f"b{l}.b2"]
-    names += ["final_g", "out_w", "out_b"]
+        names += [f"b{l}.{k}" for k in BLOCK_KEYS]
+    if cfg.head == "paper":
+        names += ["up_w", "up_b"]
+        for l in range(cfg.n_refine):
+            names += [f"r{l}.{k}" for k in BLOCK_KEYS]
+        names += ["final_g", "sp1_w", "sp1_b", "out_w", "out_b"]
+    else:
+        names += ["final_g", "out_w", "out_b"]
     return names
 
 
@@ -134,22 +155,33 @@ def weight_shapes(cfg: FDConfig) -> Dict[str, tuple]:
     """Shapes in PyTorch Linear layout ([out][in]) and the fan_in of each."""
     D, Dh, H = cfg.d_model, cfg.head_dim, cfg.n_heads
     s = {"embed_w": ((D, cfg.c_in), cfg.c_in), "embed_b": ((D,), cfg.c_in)}
-    for l in range(cfg.n_blocks):
-        s[f"b{l}.norm1_g"] = ((D,), None)
-        s[f"b{l}.wqkv"] = ((cfg.qkv_dim, D), D)
-        s[f"b{l}.bqkv"] = ((cfg.qkv_dim,), D)
-        s[f"b{l}.knorm_g"] = ((Dh,), None)
-        s[f"b{l}.vnorm_g"] = ((Dh,), None)
-        s[f"b{l}.wo"] = ((D, H * Dh), H * Dh)
-        s[f"b{l}.bo"] = ((D,), H * Dh)
-        s[f"b{l}.norm2_g"] = ((D,), None)
-        s[f"b{l}.w1"] = ((cfg.d_ff, D), D)
-        s[f"b{l}.b1"] = ((cfg.d_ff,), D)
-        s[f"b{l}.w2"] = ((D, cfg.d_ff), cfg.d_ff)
-        s[f"b{l}.b2"] = ((D,), cfg.d_ff)
+    prefixes = [f"b{l}." for l in range(cfg.n_blocks)]
+    if cfg.head == "paper":
+        prefixes += [f"r{l}." for l in range(cfg.n_refine)]
+    for p in prefixes:
+        s[p + "norm1_g"] = ((D,), None)
+        s[p + "wqkv"] = ((cfg.qkv_dim, D), D)
+        s[p + "bqkv"] = ((cfg.qkv_dim,), D)
+        s[p + "knorm_g"] = ((Dh,), None)
+        s[p + "vnorm_g"] = ((Dh,), None)
+        s[p + "wo"] = ((D, H * Dh), H * Dh)
+        s[p + "bo"] = ((D,), H * Dh)
+        s[p + "norm2_g"] = ((D,), None)
+        s[p + "w1"] = ((cfg.d_ff, D), D)
+        s[p + "b1"] = ((cfg.d_ff,), D)
+        s[p + "w2"] = ((D, cfg.d_ff), cfg.d_ff)
+        s[p + "b2"] = ((D,), cfg.d_ff)
     s["final_g"] = ((D,), None)
-    s["out_w"] = ((cfg.c_out, D), D)
-    s["out_b"] = ((cfg.c_out,), D)
+    if cfg.head == "paper":
+        s["up_w"] = ((cfg.r_t * D, D), D)
+        s["up_b"] = ((cfg.r_t * D,), D)
+        s["sp1_w"] = ((D, D), D)
+        s["sp1_b"] = ((D,), D)
+        s["out_w"] = ((cfg.c_px, D), D)
+        s["out_b"] = ((cfg.c_px,), D)
+    else:
+        s["out_w"] = ((cfg.c_out, D), D)
+        s["out_b"] = ((cfg.c_out,), D)
     return s
 
 

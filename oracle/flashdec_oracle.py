@@ -157,6 +157,13 @@ class OracleDecoder:
     The cache keeps UN-rotated keys; every step re-applies RoPE with
     window-relative temporal positions ([FD] Sec. 4.3, "Long Video
     Decoding").
+
+    With cfg.head == "paper" the output head follows [FD] Sec. 3.4: the
+    backbone output is expanded by a Linear D -> r_t D (Eq. 3) into r_t
+    sub-frames; these are streamed one after another, by the same mechanism,
+    through cfg.n_refine refinement blocks whose cache holds r_t (W+1)
+    sub-frames; each refined sub-frame goes through RMSNorm, a 2-layer MLP
+    D -> D -> C P^2 (exact GELU) and PixelShuffle by P.
     """
 
     def __init__(self, cfg, weights: Dict[str, np.ndarray]):
@@ -175,16 +182,24 @@ class OracleDecoder:
         self.t = 0
         self.cache: List[collections.deque] = [
             collections.deque() for _ in range(self.cfg.n_blocks)]
+        self.rcache: List[collections.deque] = [
+            collections.deque() for _ in range(self.cfg.n_refine if self.paper else 0)]
+
+    @property
+    def paper(self) -> bool:
+        return getattr(self.cfg, "head", "linear") == "paper"
 
     def cache_bytes(self) -> int:
         """Bytes held by the rolling caches (bounded by construction)."""
-        return sum(k.nbytes + v.nbytes for dq in self.cache for (k, v) in dq)
+        return sum(k.nbytes + v.nbytes for dq in self.cache + self.rcache for (k, v) in dq)
 
     # -- one block ---------------------------------------------------------
-    def _block(self, l: int, x: np.ndarray) -> np.ndarray:
+    def _block(self, p: str, dq: collections.deque, capacity: int,
+               x: np.ndarray) -> np.ndarray:
+        """One Transformer block (weights prefix p) for the current frame's
+        tokens x; dq is the block's cache, holding at most `capacity` frames."""
         cfg, w = self.cfg, self.w
         H, G, Dh, L = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.L_frm
-        p = f"b{l}."
         # pre-attention RMSNorm and QKV projection
         a = rms_norm(x, w[p + "norm1_g"], cfg.norm_eps)
         qkv = linear(a, w[p + "wqkv"], w[p + "bqkv"])
@@ -194,10 +209,9 @@ class OracleDecoder:
         if cfg.kv_norm:
             k = rms_norm(k, w[p + "knorm_g"], cfg.norm_eps)
             v = rms_norm(v, w[p + "vnorm_g"], cfg.norm_eps)
-        # append to the cache, evict the oldest beyond W+1 frames
-        dq = self.cache[l]
+        # append to the cache, evict the oldest beyond its capacity
         dq.append((k, v))
-        if len(dq) > cfg.window + 1:
+        if len(dq) > capacity:
             dq.popleft()
         n_win = len(dq)
         # window-relative temporal positions: oldest frame 0, current n_win-1
@@ -227,20 +241,41 @@ class OracleDecoder:
         return linear(u, self.w["embed_w"], self.w["embed_b"])
 
     def head(self, x: np.ndarray) -> np.ndarray:
-        """Final RMSNorm, Linear D -> C r_t P^2, unpatchify."""
+        """Linear head: final RMSNorm, Linear D -> C r_t P^2, unpatchify."""
         cfg = self.cfg
         y = linear(rms_norm(x, self.w["final_g"], cfg.norm_eps),
                    self.w["out_w"], self.w["out_b"])
         return unpatchify(y, cfg.out_ch, cfg.r_t, cfg.px_per_token,
                           cfg.tok_h, cfg.tok_w)
 
+    def spatial(self, xs: np.ndarray) -> np.ndarray:
+        """Paper head, Step 3 ([FD] Sec. 3.4): RMSNorm, MLP D -> D -> C P^2,
+        PixelShuffle by P -> one pixel frame [C][tok_h P][tok_w P]."""
+        cfg, w = self.cfg, self.w
+        h = gelu(linear(rms_norm(xs, w["final_g"], cfg.norm_eps), w["sp1_w"], w["sp1_b"]))
+        y = linear(h, w["out_w"], w["out_b"])
+        return unpatchify(y, cfg.out_ch, 1, cfg.px_per_token, cfg.tok_h,
+                          cfg.tok_w)[:, 0]
+
     def decode_frame(self, z_t: np.ndarray) -> np.ndarray:
         """One streaming step: latent frame t -> r_t pixel frames."""
+        cfg = self.cfg
         x = self.embed(z_t)
-        for l in range(self.cfg.n_blocks):
-            x = self._block(l, x)
+        for l in range(cfg.n_blocks):
+            x = self._block(f"b{l}.", self.cache[l], cfg.window + 1, x)
         self.t += 1
-        return self.head(x)
+        if not self.paper:
+            return self.head(x)
+        # temporal upsampling (Eq. 3): channels [tau D, (tau+1) D) -> sub-frame tau
+        up = linear(x, self.w["up_w"], self.w["up_b"])
+        D = cfg.d_model
+        frames = []
+        for tau in range(cfg.r_t):
+            xs = up[:, tau * D:(tau + 1) * D]
+            for l in range(cfg.n_refine):
+                xs = self._block(f"r{l}.", self.rcache[l], cfg.r_t * (cfg.window + 1), xs)
+            frames.append(self.spatial(xs))
+        return np.stack(frames, axis=1)                  # [C][r_t][H][W]
 
     def window_frames(self, l: int):
         """Frame indices currently held by block l's cache, oldest first."""
@@ -266,6 +301,45 @@ def decode_video(cfg, weights, z: np.ndarray,
 # Full-sequence forward with a brute-force block-windowed mask
 # --------------------------------------------------------------------------
 
+def _masked_block(cfg, w, p, x, tau, row, col, allowed):
+    """One block over a whole token sequence with a boolean attention mask
+    (allowed[a, b]: query token a may see key token b); absolute positions."""
+    H, G, Dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    S = x.shape[0]
+    a = rms_norm(x, w[p + "norm1_g"], cfg.norm_eps)
+    qkv = linear(a, w[p + "wqkv"], w[p + "bqkv"])
+    q = qkv[:, :H * Dh].reshape(S, H, Dh)
+    k = qkv[:, H * Dh:(H + G) * Dh].reshape(S, G, Dh)
+    v = qkv[:, (H + G) * Dh:].reshape(S, G, Dh)
+    if cfg.kv_norm:
+        k = rms_norm(k, w[p + "knorm_g"], cfg.norm_eps)
+        v = rms_norm(v, w[p + "vnorm_g"], cfg.norm_eps)
+    o = np.empty((S, H, Dh))
+    for h in range(H):
+        g = h // (H // G)
+        qh = rope_3d(q[:, h], tau, row, col, cfg.rope_theta)
+        kh = rope_3d(k[:, g], tau, row, col, cfg.rope_theta)
+        sc = (qh @ kh.T) / np.sqrt(Dh)
+        sc = np.where(allowed, sc, -np.inf)
+        sc = sc - sc.max(axis=-1, keepdims=True)
+        pr = np.exp(sc)
+        pr = pr / pr.sum(axis=-1, keepdims=True)
+        o[:, h] = pr @ v[:, g]
+    x = x + linear(o.reshape(S, H * Dh), w[p + "wo"], w[p + "bo"])
+    a = rms_norm(x, w[p + "norm2_g"], cfg.norm_eps)
+    return x + linear(gelu(linear(a, w[p + "w1"], w[p + "b1"])), w[p + "w2"], w[p + "b2"])
+
+
+def _window_mask(frame_of, span):
+    """allowed[a, b] = frame_of[b] in [frame_of[a] - span + 1, frame_of[a]]."""
+    S = frame_of.shape[0]
+    allowed = np.zeros((S, S), dtype=bool)
+    for a in range(S):
+        for b in range(S):
+            allowed[a, b] = (frame_of[a] - span + 1 <= frame_of[b] <= frame_of[a])
+    return allowed
+
+
 def full_sequence(cfg, weights: Dict[str, np.ndarray],
                   z: np.ndarray) -> np.ndarray:
     """One forward over all T' L_frm tokens at once.
@@ -275,50 +349,43 @@ def full_sequence(cfg, weights: Dict[str, np.ndarray],
     sequence goes through one pass and a materialised mask restricts each
     query of frame t to key frames t-W .. t (the sliding-window pattern of
     [FD] Sec. 3.3, "Attention Pattern"). RoPE uses ABSOLUTE frame indices.
-    Only for tiny inputs: the mask is [T' L][T' L].
+    With the paper head, the r_t T' sub-frames go through the refinement
+    blocks the same way (sub-frame s sees sub-frames s - r_t (W+1) + 1 .. s).
+    Only for tiny inputs: the masks are [T' L][T' L] and [r_t T' L]^2.
     """
     w = {k: np.asarray(v, dtype=np.float64) for k, v in weights.items()}
     T = z.shape[0]
-    H, G, Dh, L = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.L_frm
-    S = T * L
+    D, L = cfg.d_model, cfg.L_frm
     frame_of = np.repeat(np.arange(T), L)                 # frame of each token
     n = np.tile(np.arange(L), T)
     row = (n // cfg.tok_w).astype(np.float64)
     col = (n % cfg.tok_w).astype(np.float64)
-    tau = frame_of.astype(np.float64)
-    allowed = np.zeros((S, S), dtype=bool)
-    for a in range(S):
-        for b in range(S):
-            allowed[a, b] = (frame_of[a] - cfg.window <= frame_of[b] <= frame_of[a])
+    allowed = _window_mask(frame_of, cfg.window + 1)
 
     x = np.concatenate([linear(patchify(z[t].astype(np.float64), cfg.patch),
                                w["embed_w"], w["embed_b"]) for t in range(T)])
     for l in range(cfg.n_blocks):
-        p = f"b{l}."
-        a = rms_norm(x, w[p + "norm1_g"], cfg.norm_eps)
-        qkv = linear(a, w[p + "wqkv"], w[p + "bqkv"])
-        q = qkv[:, :H * Dh].reshape(S, H, Dh)
-        k = qkv[:, H * Dh:(H + G) * Dh].reshape(S, G, Dh)
-        v = qkv[:, (H + G) * Dh:].reshape(S, G, Dh)
-        if cfg.kv_norm:
-            k = rms_norm(k, w[p + "knorm_g"], cfg.norm_eps)
-            v = rms_norm(v, w[p + "vnorm_g"], cfg.norm_eps)
-        o = np.empty((S, H, Dh))
-        for h in range(H):
-            g = h // (H // G)
-            qh = rope_3d(q[:, h], tau, row, col, cfg.rope_theta)
-            kh = rope_3d(k[:, g], tau, row, col, cfg.rope_theta)
-            sc = (qh @ kh.T) / np.sqrt(Dh)
-            sc = np.where(allowed, sc, -np.inf)
-            sc = sc - sc.max(axis=-1, keepdims=True)
-            pr = np.exp(sc)
-            pr = pr / pr.sum(axis=-1, keepdims=True)
-            o[:, h] = pr @ v[:, g]
-        x = x + linear(o.reshape(S, H * Dh), w[p + "wo"], w[p + "bo"])
-        a = rms_norm(x, w[p + "norm2_g"], cfg.norm_eps)
-        x = x + linear(gelu(linear(a, w[p + "w1"], w[p + "b1"])),
-                       w[p + "w2"], w[p + "b2"])
-    y = linear(rms_norm(x, w["final_g"], cfg.norm_eps), w["out_w"], w["out_b"])
-    return np.stack([unpatchify(y[t * L:(t + 1) * L], cfg.out_ch, cfg.r_t,
-                                cfg.px_per_token, cfg.tok_h, cfg.tok_w)
-                     for t in range(T)])
+        x = _masked_block(cfg, w, f"b{l}.", x, frame_of.astype(np.float64), row, col, allowed)
+    if getattr(cfg, "head", "linear") != "paper":
+        y = linear(rms_norm(x, w["final_g"], cfg.norm_eps), w["out_w"], w["out_b"])
+        return np.stack([unpatchify(y[t * L:(t + 1) * L], cfg.out_ch, cfg.r_t,
+                                    cfg.px_per_token, cfg.tok_h, cfg.tok_w)
+                         for t in range(T)])
+    # paper head: sub-frame s = t r_t + tau takes channels [tau D, (tau+1) D)
+    up = linear(x, w["up_w"], w["up_b"]).reshape(T, L, cfg.r_t, D)
+    xs = up.transpose(0, 2, 1, 3).reshape(T * cfg.r_t * L, D)
+    sub_of = np.repeat(np.arange(T * cfg.r_t), L)
+    n = np.tile(np.arange(L), T * cfg.r_t)
+    row = (n // cfg.tok_w).astype(np.float64)
+    col = (n % cfg.tok_w).astype(np.float64)
+    allowed = _window_mask(sub_of, cfg.r_t * (cfg.window + 1))
+    for l in range(cfg.n_refine):
+        xs = _masked_block(cfg, w, f"r{l}.", xs, sub_of.astype(np.float64), row, col, allowed)
+    h = gelu(linear(rms_norm(xs, w["final_g"], cfg.norm_eps), w["sp1_w"], w["sp1_b"]))
+    y = linear(h, w["out_w"], w["out_b"])
+    out = np.empty((T,) + tuple(cfg.out_shape))
+    for s in range(T * cfg.r_t):
+        t, tau = divmod(s, cfg.r_t)
+        out[t, :, tau] = unpatchify(y[s * L:(s + 1) * L], cfg.out_ch, 1, cfg.px_per_token,
+                                    cfg.tok_h, cfg.tok_w)[:, 0]
+    return out

@@ -347,3 +347,103 @@ def test_zero_query_weights_give_window_mean_of_values():
         for s in range(t + 1):
             out = dec2.decode_frame(z[s])
         np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# The paper's output head ([FD] Sec. 3.4)
+# --------------------------------------------------------------------------
+
+def _paper(**kw):
+    base = dict(head="paper", n_refine=2, window=1, n_blocks=1)
+    base.update(kw)
+    return _small(**base)
+
+
+def _torch_library_paper_decoder(cfg, weights, z):
+    """Paper head on top of the torch-library backbone: F.linear for the
+    temporal upsampling, the same masked library block for the refinement
+    blocks over all r_t T' sub-frames (absolute sub-frame positions),
+    F.rms_norm + F.linear + F.gelu + F.linear, F.pixel_shuffle."""
+    W = {k: torch.from_numpy(np.asarray(v, np.float64)) for k, v in weights.items()}
+    T, L, D, rt = z.shape[0], cfg.L_frm, cfg.d_model, cfg.r_t
+    H, G, Dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    parts = [Dh // 4, 3 * Dh // 8, Dh - Dh // 4 - 3 * Dh // 8]
+
+    def rope(t, pos_axes):
+        chunks, lo = [], 0
+        for d, pos in zip(parts, pos_axes):
+            c = torch.view_as_complex(t[..., lo:lo + d].reshape(*t.shape[:2], d // 2, 2).contiguous())
+            freq = cfg.rope_theta ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+            c = c * torch.polar(torch.ones(()).double(), pos[:, None, None] * freq)
+            chunks.append(torch.view_as_real(c).reshape(*t.shape[:2], d))
+            lo += d
+        return torch.cat(chunks, -1)
+
+    def block(x, p, fr, span):
+        n = torch.arange(x.shape[0]) % L
+        pos_axes = [fr.double(), (n // cfg.tok_w).double(), (n % cfg.tok_w).double()]
+        mask = (fr[None, :] <= fr[:, None]) & (fr[None, :] > fr[:, None] - span)
+        a = F.rms_norm(x, (D,), W[p + "norm1_g"], eps=cfg.norm_eps)
+        q, k, v = F.linear(a, W[p + "wqkv"], W[p + "bqkv"]).split([H * Dh, G * Dh, G * Dh], -1)
+        q, k, v = q.view(-1, H, Dh), k.view(-1, G, Dh), v.view(-1, G, Dh)
+        if cfg.kv_norm:
+            k = F.rms_norm(k, (Dh,), W[p + "knorm_g"], eps=cfg.norm_eps)
+            v = F.rms_norm(v, (Dh,), W[p + "vnorm_g"], eps=cfg.norm_eps)
+        q, k = rope(q, pos_axes), rope(k, pos_axes)
+        k, v = k.repeat_interleave(H // G, 1), v.repeat_interleave(H // G, 1)
+        o = F.scaled_dot_product_attention(q.transpose(0, 1), k.transpose(0, 1),
+                                           v.transpose(0, 1), attn_mask=mask)
+        x = x + F.linear(o.transpose(0, 1).reshape(-1, H * Dh), W[p + "wo"], W[p + "bo"])
+        a = F.rms_norm(x, (D,), W[p + "norm2_g"], eps=cfg.norm_eps)
+        return x + F.linear(F.gelu(F.linear(a, W[p + "w1"], W[p + "b1"])), W[p + "w2"], W[p + "b2"])
+
+    zt = torch.from_numpy(np.asarray(z, np.float64))
+    toks = F.pixel_unshuffle(zt, cfg.patch).flatten(2).transpose(1, 2).reshape(T * L, cfg.c_in)
+    x = F.linear(toks, W["embed_w"], W["embed_b"])
+    fr = torch.arange(T).repeat_interleave(L)
+    for l in range(cfg.n_blocks):
+        x = block(x, f"b{l}.", fr, cfg.window + 1)
+    up = F.linear(x, W["up_w"], W["up_b"]).view(T, L, rt, D).permute(0, 2, 1, 3).reshape(-1, D)
+    sub = torch.arange(T * rt).repeat_interleave(L)
+    for l in range(cfg.n_refine):
+        up = block(up, f"r{l}.", sub, rt * (cfg.window + 1))
+    h = F.gelu(F.linear(F.rms_norm(up, (D,), W["final_g"], eps=cfg.norm_eps), W["sp1_w"], W["sp1_b"]))
+    y = F.linear(h, W["out_w"], W["out_b"]).view(T * rt, cfg.tok_h, cfg.tok_w, cfg.c_px)
+    px = F.pixel_shuffle(y.permute(0, 3, 1, 2), cfg.px_per_token)      # [T rt][C][H][W]
+    return px.view(T, rt, *px.shape[1:]).permute(0, 2, 1, 3, 4).numpy()
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(n_heads=4, n_kv_heads=2), dict(window=0, n_refine=1)])
+def test_paper_head_streaming_matches_torch_library_composition(kw):
+    cfg = _paper(**kw)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg, frames=4)
+    got = oracle.decode_video(cfg, w, z)
+    ref = _torch_library_paper_decoder(cfg, w, z)
+    assert got.shape == ref.shape == (4,) + tuple(cfg.out_shape)
+    np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-10)
+
+
+def test_paper_head_streaming_equals_masked_full_sequence():
+    # 4 latent frames -> 16 sub-frames through a refinement window of
+    # r_t (W+1) = 8 sub-frames: eviction in the refinement cache is covered
+    cfg = _paper(grid_h=2, grid_w=4)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg, frames=4)
+    s = oracle.decode_video(cfg, w, z)
+    f = oracle.full_sequence(cfg, w, z)
+    assert _rel(s, f) <= 1e-12
+
+
+def test_paper_head_causality_and_cache_bound():
+    cfg = _paper()
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg, frames=5)
+    base = oracle.decode_video(cfg, w, z)
+    pert = oracle.decode_video(cfg, w, fd_synth.perturb_frame(z, 3))
+    np.testing.assert_array_equal(pert[:3], base[:3])
+    assert not np.array_equal(pert[3], base[3])
+    dec = oracle.OracleDecoder(cfg, w)
+    for t in range(5):
+        dec.decode_frame(z[t])
+        assert all(len(dq) == min(cfg.r_t * (t + 1), cfg.r_t * (cfg.window + 1)) for dq in dec.rcache)
