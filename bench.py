@@ -49,29 +49,65 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def is_paper(cfg) -> bool:
+    return getattr(cfg, "head", "linear") == "paper"
+
+
 def describe(cfg) -> str:
+    head = (f"paper head (upsample x{cfg.r_t}, {cfg.n_refine} refinement blocks over "
+            f"{cfg.r_t * (cfg.window + 1)} sub-frames, spatial MLP)" if is_paper(cfg)
+            else "linear head")
     return (f"{cfg.name}: latent {cfg.latent_ch}ch {cfg.grid_h}x{cfg.grid_w}, patch {cfg.patch} "
-            f"({cfg.L_frm} tokens/frame), d={cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}, "
-            f"{cfg.n_blocks} blocks, MLP {cfg.mlp_ratio}x, W={cfg.window}; each latent frame -> "
+            f"({cfg.L_frm} tokens/frame), d={cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}"
+            f" / {cfg.n_kv_heads} KV groups, {cfg.n_blocks} blocks, MLP {cfg.mlp_ratio}x, "
+            f"W={cfg.window}, {head}; each latent frame -> "
             f"{cfg.out_ch}x{cfg.r_t}x{cfg.out_shape[2]}x{cfg.out_shape[3]} px")
 
 
-def flops_per_frame(cfg, n_valid=None):
-    """Algorithmic FLOPs of one latent frame (2 per MAC). n_valid: frames in
-    the window (default: full, W+1)."""
-    L, D, nb = cfg.L_frm, cfg.d_model, cfg.n_blocks
-    nv = cfg.window + 1 if n_valid is None else n_valid
-    qkv = 2 * L * D * cfg.qkv_dim
-    oproj = 2 * L * cfg.n_heads * cfg.head_dim * D
-    mlp = 2 * 2 * L * D * cfg.d_ff
-    attn = 4 * L * (nv * L) * cfg.n_heads * cfg.head_dim
-    gemm = nb * (qkv + oproj + mlp) + 2 * L * cfg.c_in * D + 2 * L * D * cfg.c_out
-    return gemm + nb * attn, nb * attn
-
-
 def attn_flops_per_launch(cfg):
-    L = cfg.L_frm
-    return 4 * L * ((cfg.window + 1) * L) * cfg.n_heads * cfg.head_dim
+    """FLOPs of each attention launch of one steady-state frame, in launch
+    order: the backbone blocks (window of W+1 frames), then with the paper
+    head r_t x n_refine refinement launches (window of r_t (W+1) sub-frames)."""
+    L, hd = cfg.L_frm, cfg.n_heads * cfg.head_dim
+    out = [4 * L * ((cfg.window + 1) * L) * hd] * cfg.n_blocks
+    if is_paper(cfg):
+        out += [4 * L * (cfg.r_t * (cfg.window + 1) * L) * hd] * (cfg.r_t * cfg.n_refine)
+    return out
+
+
+def kind_flops(cfg):
+    """FLOPs of one launch of each GEMM kind (2 per MAC)."""
+    L, D = cfg.L_frm, cfg.d_model
+    f = {"qkv": 2 * L * D * cfg.qkv_dim, "oproj": 2 * L * cfg.n_heads * cfg.head_dim * D,
+         "mlp_up": 2 * L * D * cfg.d_ff, "mlp_down": 2 * L * D * cfg.d_ff,
+         "embed": 2 * L * cfg.c_in * D}
+    if is_paper(cfg):
+        f.update(upsample=2 * L * D * cfg.r_t * D, spatial=2 * L * D * D,
+                 final=2 * L * D * cfg.c_px)
+    else:
+        f["final"] = 2 * L * D * cfg.c_out
+    return f
+
+
+def kernels_per_frame(cfg) -> int:
+    n = 2 + 5 * cfg.n_blocks                            # step_begin, embed, backbone
+    if is_paper(cfg):
+        return n + 1 + cfg.r_t * (5 * cfg.n_refine + 2)  # upsample, refinement, spatial MLP
+    return n + 1                                        # final
+
+
+def flops_per_frame(cfg):
+    """Algorithmic FLOPs of one steady-state latent frame; returns (total,
+    attention part)."""
+    k = kind_flops(cfg)
+    block = k["qkv"] + k["oproj"] + k["mlp_up"] + k["mlp_down"]
+    attn = sum(attn_flops_per_launch(cfg))
+    gemm = k["embed"] + cfg.n_blocks * block
+    if is_paper(cfg):
+        gemm += k["upsample"] + cfg.r_t * (cfg.n_refine * block + k["spatial"] + k["final"])
+    else:
+        gemm += k["final"]
+    return gemm + attn, attn
 
 
 def file_sha(path):
@@ -166,26 +202,39 @@ def replica_throughput(r_t, frames_all_ranks, max_ms):
 
 
 # ------------------------------------------------------------------ oracle
+def one_block_weights(cfg, weights):
+    """Weights of the same decoder with its first backbone block only."""
+    return {k: v for k, v in weights.items()
+            if not (k.startswith("b") and not k.startswith("b0."))}
+
+
+def time_backbone_block(dec, z_t):
+    """Seconds of one backbone block of the oracle on a full window (the
+    block's cache is left as it was)."""
+    import collections
+    x = dec.embed(z_t)
+    dq = collections.deque(dec.cache[0])
+    t0 = time.perf_counter()
+    dec._block("b0.", dq, dec.cfg.window + 1, x)
+    return time.perf_counter() - t0
+
+
 def oracle_sample_seconds(cfg, weights_1blk, z):
-    """Time the CPU oracle on a bounded sample: frames 0..W of a 1-block
-    decoder at the workload's full width (untimed set-up), then frame W+1
-    (full window) timed, plus the embedding and head timed separately.
-    Returns (seconds per latent frame of the full-depth decoder, detail)."""
+    """Time the CPU oracle on a bounded sample: frames 0..W of a decoder with
+    one backbone block at the workload's full width (untimed set-up), then
+    frame W+1 (full window, head included) timed, and one more backbone block
+    timed alone. Returns (seconds per latent frame of the full-depth decoder,
+    detail) = frame + (n_blocks - 1) x block."""
     import oracle
-    cfg1 = cfg.replace(n_blocks=1)
-    dec = oracle.OracleDecoder(cfg1, weights_1blk)
+    dec = oracle.OracleDecoder(cfg.replace(n_blocks=1), weights_1blk)
     for t in range(cfg.window + 1):
         dec.decode_frame(z[t])
     t0 = time.perf_counter()
     dec.decode_frame(z[cfg.window + 1])
     t_one = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    x = dec.embed(z[0])
-    dec.head(x)
-    t_eh = time.perf_counter() - t0
-    t_block = max(t_one - t_eh, 1e-9)
-    per_frame = t_eh + cfg.n_blocks * t_block
-    return per_frame, dict(t_block_s=t_block, t_embed_head_s=t_eh)
+    t_block = time_backbone_block(dec, z[0])
+    per_frame = t_one + (cfg.n_blocks - 1) * t_block
+    return per_frame, dict(t_block_s=t_block, t_frame_1blk_s=t_one)
 
 
 def blas_threads():
@@ -202,7 +251,7 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     cfg = fd_synth.CONFIGS[args.config]
-    w1 = fd_synth.make_weights(cfg.replace(n_blocks=1))
+    w1 = one_block_weights(cfg, fd_synth.make_weights(cfg))
     frames = args.warmup + args.steps + cfg.window + 2
     z = fd_synth.make_latents(cfg, frames=frames)
     import oracle
@@ -212,20 +261,18 @@ def run_reference(args):
     t = cfg.window + 1
     for _ in range(args.warmup):
         dec.decode_frame(z[t]); t += 1
-    t0 = time.perf_counter()
-    dec.head(dec.embed(z[0]))
-    t_eh = time.perf_counter() - t0
+    t_block = time_backbone_block(dec, z[0])
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
         dec.decode_frame(z[t]); t += 1
         times.append(time.perf_counter() - t0)
-    t_block = max(float(np.mean(times)) - t_eh, 1e-9)
-    per_frame = t_eh + cfg.n_blocks * t_block
+    per_frame = float(np.mean(times)) + (cfg.n_blocks - 1) * t_block
     value = cfg.r_t / per_frame
-    sample = (f"each step: one full-window latent frame of a 1-block decoder at the workload's "
-              f"full width ({cfg.L_frm} tokens, {(cfg.window + 1) * cfg.L_frm}-token window); "
-              f"per-frame time = embed+head + {cfg.n_blocks} x block time")
+    sample = (f"each step: one full-window latent frame of the decoder with 1 backbone block at "
+              f"the workload's full width ({cfg.L_frm} tokens, {(cfg.window + 1) * cfg.L_frm}-"
+              f"token window), head included; per-frame time = that + {cfg.n_blocks - 1} x one "
+              f"backbone block ({t_block:.2f} s, timed once)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_frame * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -293,7 +340,7 @@ def run_flashdec(args):
     lat_ms = [a.elapsed_time(b) for a, b in ev]
     frames_all = sum_over_ranks(dist, args.steps)
     value = replica_throughput(cfg.r_t, frames_all, total_ms)
-    kernels_per_frame = 2 + 5 * cfg.n_blocks + 1   # step_begin, embed, blocks, final
+    launches = kernels_per_frame(cfg)
 
     # ---- end to end: host buffers through fd_decode_frame_host
     lat_h = [torch.from_numpy(z[t]).to(td).pin_memory() for t in range(n_frames)]
@@ -338,8 +385,9 @@ def run_flashdec(args):
     # ---- roofline of the dominant kernel (attention) and of the whole step
     peaks, peak_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    attn_ms = float(np.mean(attn_launch_ms))
-    attn_tf = attn_flops_per_launch(cfg) / (attn_ms * 1e-3) / 1e12
+    attn_fl = attn_flops_per_launch(cfg)
+    assert len(attn_fl) == len(attn_launch_ms)
+    attn_tf = sum(attn_fl) / (sum(attn_launch_ms) * 1e-3) / 1e12
     src = os.path.join(ROOT, "streaming_transformer_video_b200", "csrc", "fd_attn_tc.cuh")
     traffic = NCU_ATTN_TRAFFIC.get((args.config, file_sha(src)))
     step_flops, _ = flops_per_frame(cfg)
@@ -347,14 +395,14 @@ def run_flashdec(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        w1 = {k: v for k, v in weights.items() if not k.startswith("b") or k.startswith("b0.")}
-        per_frame, detail = oracle_sample_seconds(cfg, w1, z)
+        per_frame, detail = oracle_sample_seconds(cfg, one_block_weights(cfg, weights), z)
         cpu = {"value": cfg.r_t / per_frame, "unit": UNIT, "cores": blas_threads(),
                "kind": "oracle",
-               "sample": (f"frame {cfg.window + 1} (full {cfg.window + 1}-frame window) of a "
-                          f"1-block decoder at full width, after frames 0..{cfg.window} "
-                          f"untimed; per-frame time = embed+head ({detail['t_embed_head_s']:.2f} s)"
-                          f" + {cfg.n_blocks} x block ({detail['t_block_s']:.2f} s)")}
+               "sample": (f"frame {cfg.window + 1} (full {cfg.window + 1}-frame window) of the "
+                          f"decoder with 1 backbone block at full width, head included "
+                          f"({detail['t_frame_1blk_s']:.2f} s), after frames 0..{cfg.window} "
+                          f"untimed; per-frame time = that + {cfg.n_blocks - 1} x one backbone "
+                          f"block ({detail['t_block_s']:.2f} s)")}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -376,18 +424,17 @@ def run_flashdec(args):
         "kernels_ms": {k: float(np.mean(v)) for k, v in kern.items()},
         "kernels_tflops": {},
         "clocks": clk,
-        "gpu_launches": kernels_per_frame * args.steps,
+        "gpu_launches": launches * args.steps,
         "device_bytes": dev_bytes,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
     }
-    L, D = cfg.L_frm, cfg.d_model
-    per_kind_flops = {"qkv": 2 * L * D * cfg.qkv_dim, "oproj": 2 * L * cfg.n_heads * cfg.head_dim * D,
-                      "mlp_up": 2 * L * D * cfg.d_ff, "mlp_down": 2 * L * D * cfg.d_ff,
-                      "final": 2 * L * D * cfg.c_out, "attn": attn_flops_per_launch(cfg)}
-    for k, f in per_kind_flops.items():
-        if k in line["kernels_ms"]:
+    for k, f in kind_flops(cfg).items():
+        if k in kern and k != "embed":
             line["kernels_tflops"][k] = f / (line["kernels_ms"][k] * 1e-3) / 1e12
+    # attention launches of the last frame of the breakdown pass, in launch order
+    per_frame_attn = kern["attn"][-len(attn_fl):]
+    line["kernels_tflops"]["attn"] = sum(attn_fl) / (sum(per_frame_attn) * 1e-3) / 1e12
     if cpu is not None:
         line["cpu_baseline"] = cpu
     dec.close()

@@ -128,6 +128,16 @@ CONFIGS: Dict[str, FDConfig] = {
     # (48ch, 30x52 grid, 1560 tokens), 7 latent frames.
     "xl_480p_wan22": FDConfig("xl_480p_wan22", 48, 30, 52, 1, 1536, 24, 3, 64,
                               20, 4, 1, 3, 4, 16, 1, "bf16", 7),
+    # FlashDecoder-XL with the paper's own head (Sec. 3.4): the XL backbone
+    # above, temporal upsampling by r_t = 4, 2 refinement blocks over a window
+    # of r_t (W+1) = 8 sub-frames, RMSNorm + MLP 1536 -> 1536 -> 3*16*16 and
+    # PixelShuffle; 480p and 720p Wan2.2 latents.
+    "xl_480p_wan22_paper": FDConfig("xl_480p_wan22_paper", 48, 30, 52, 1, 1536, 24, 3,
+                                    64, 20, 4, 1, 3, 4, 16, 1, "bf16", 7,
+                                    head="paper", n_refine=2),
+    "xl_720p_wan22_paper": FDConfig("xl_720p_wan22_paper", 48, 45, 80, 1, 1536, 24, 3,
+                                    64, 20, 4, 1, 3, 4, 16, 1, "bf16", 7,
+                                    head="paper", n_refine=2),
 }
 
 

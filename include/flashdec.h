@@ -8,7 +8,12 @@
  * Transformer block computes new keys and values, appends them to a rolling
  * cache and evicts the oldest frame (Eq. 2), and the frame's queries attend,
  * with no mask, to every cached token. A final projection turns each token
- * into r_t pixel frames of P x P pixels (Sec. 3.4, Step 3).
+ * into r_t pixel frames of P x P pixels (Sec. 3.4, Step 3). With head_mode 1
+ * the output head is the paper's own (Sec. 3.4): a Linear D -> r_t D splits
+ * each latent frame into r_t sub-frames (Eq. 3), refinement blocks stream
+ * those sub-frames one after another with the same rolling-cache mechanism
+ * (ring of r_t (W+1) sub-frames), and a 2-layer MLP + PixelShuffle turns each
+ * refined sub-frame into one pixel frame.
  *
  * Conventions of this library:
  *   - W (fd_config.window) counts PAST latent frames. The cache keeps the
@@ -78,6 +83,13 @@ typedef struct {
                             fd_last_step_kernel_ms: 0 off; 1 around every
                             kernel; 2 around each attention launch only (the
                             dominant kernel; negligible overhead)                */
+  int32_t head_mode;     /* 0: final RMSNorm + Linear D -> C r_t P^2 + unpatchify.
+                            1: the paper's head (Sec. 3.4): Linear D -> r_t D
+                            (Eq. 3) into r_t sub-frames, streamed through
+                            n_refine refinement blocks with a cache of r_t (W+1)
+                            sub-frames, then RMSNorm, Linear D -> D, GELU,
+                            Linear D -> C P^2 and PixelShuffle per sub-frame    */
+  int32_t n_refine;      /* refinement blocks (head_mode 1; 1 .. 8)              */
 } fd_config;
 
 /*
@@ -94,6 +106,14 @@ typedef struct {
  *            w1 [mlp_ratio D][D], b1; w2 [D][mlp_ratio D], b2 [D]
  *   final_g [D]; out_w [C r_t P^2][D] with output channel order
  *            (c, tau, dy, dx); out_b [C r_t P^2]
+ * With head_mode 1 the per-block arrays hold n_blocks + n_refine entries
+ * (backbone blocks, then refinement blocks), final_g is the RMSNorm gain
+ * before the spatial MLP, and:
+ *   up_w [r_t D][D], up_b [r_t D]       temporal upsampling; output channels
+ *            [tau D, (tau+1) D) form sub-frame tau
+ *   sp1_w [D][D], sp1_b [D]             first spatial MLP layer
+ *   out_w [C P^2][D], out_b [C P^2]     second layer, channel order (c, dy, dx)
+ * (up_w .. sp1_b are ignored with head_mode 0.)
  */
 typedef struct {
   const float *embed_w, *embed_b;
@@ -102,6 +122,7 @@ typedef struct {
   const float *const *wo, *const *bo, *const *norm2_g;
   const float *const *w1, *const *b1, *const *w2, *const *b2;
   const float *final_g, *out_w, *out_b;
+  const float *up_w, *up_b, *sp1_w, *sp1_b;
 } fd_weights;
 
 /*
@@ -169,13 +190,15 @@ FD_API fd_status_t fd_frame_index(fd_handle* h, int64_t* t_out);
 /* Device bytes held by the handle (weights, ring cache, scratch, staging). */
 FD_API fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out);
 
-/* Bytes of the ring cache alone: n_blocks * 2 * G * (W+1) L_frm * D_h * elt. */
+/* Bytes of the ring caches alone: n_blocks * 2 * G * (W+1) L_frm * D_h * elt,
+ * plus n_refine * 2 * G * r_t (W+1) L_frm * D_h * elt with head_mode 1. */
 FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 
 /*
- * Test/debug: copy ring slot `slot` of block `block` to host memory as fp32
- * [G][L_frm][D_h]. kv = 0 reads keys (stored after KV-norm and RoPE at the
- * frame's absolute index), kv = 1 reads values (after KV-norm). Synchronous.
+ * Test/debug: copy ring slot `slot` of backbone block `block` to host memory
+ * as fp32 [G][L_frm][D_h]. kv = 0 reads keys (stored after KV-norm and RoPE
+ * at the frame's absolute index), kv = 1 reads values (after KV-norm).
+ * Synchronous.
  */
 FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
 
@@ -187,9 +210,13 @@ FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv,
  * *n_out = number of timed kernels per frame. Pass cap = 0 to query *n_out
  * only. Each replay of the frame graph overwrites the previous frame's times.
  */
+/* With head_mode 1 a frame runs, after the backbone: UPSAMPLE once, then per
+ * sub-frame the refinement blocks' QKV .. MLP_DOWN kernels, SPATIAL (first
+ * MLP layer) and FINAL (second layer + PixelShuffle). */
 typedef enum {
   FD_K_STEP_BEGIN = 0, FD_K_EMBED = 1, FD_K_QKV = 2, FD_K_ATTN = 3,
-  FD_K_OPROJ = 4, FD_K_MLP_UP = 5, FD_K_MLP_DOWN = 6, FD_K_FINAL = 7
+  FD_K_OPROJ = 4, FD_K_MLP_UP = 5, FD_K_MLP_DOWN = 6, FD_K_FINAL = 7,
+  FD_K_UPSAMPLE = 8, FD_K_SPATIAL = 9
 } fd_kernel_kind;
 FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out,
                                    int32_t cap, int32_t* n_out);

@@ -9,7 +9,12 @@
 // Per-frame kernel sequence (bf16 configuration, all sm_100a):
 //   step_begin -> embed -> n_blocks x [QKV GEMM (+norm, KV-norm, RoPE, ring
 //   write) -> attention -> O-proj GEMM (+residual) -> MLP-up GEMM (+GELU) ->
-//   MLP-down GEMM (+residual)] -> final GEMM (+norm, unpatchify)
+//   MLP-down GEMM (+residual)] -> head
+// Linear head: final GEMM (+norm, unpatchify).
+// Paper head (Sec. 3.4): upsample GEMM (Eq. 3, one launch for all r_t
+//   sub-frames) -> for each sub-frame tau in order: n_refine x [the five block
+//   kernels on sub-frame tau, refinement ring] -> spatial GEMM (+norm, GELU)
+//   -> final GEMM (PixelShuffle into pixel frame tau).
 // The fp32 configuration runs the same sequence with CUDA-core kernels.
 #include <cudaTypedefs.h>
 
@@ -122,6 +127,33 @@ struct KernelLaunch {
   int kind;
 };
 
+// Where one Transformer block reads and writes: its residual stream (one
+// latent frame, or one sub-frame of the paper head) and its ring cache.
+struct BlockIO {
+  float* x32;               // [L][D] fp32 residual stream
+  void* xb;                 // [L][D] storage-type copy (A operand)
+  float* ssq;               // [L][D/32] sums of squares of x32
+  const CUtensorMap* tm_x;  // map of xb (bf16 path)
+  void* kc;                 // ring keys   [layers][G][kv_rows][Dh]
+  void* vtc;                // ring values [layers][G][Dh][vt_pitch]
+  int kv_rows, vt_pitch;
+  const CUtensorMap* tm_k;  // maps over all layers of kc / vtc (bf16 path)
+  const CUtensorMap* tm_v;
+  int layer;                // this block's layer inside kc / vtc
+  const FrameState* fs;     // frame state of the streamed (sub-)frame
+};
+
+// A kernel node that writes the caller's pixel buffer (patched per call).
+struct OutNode {
+  cudaGraphNode_t node = nullptr;
+  KernelLaunch launch{};
+  EpiParams p{};
+  CUtensorMap tmA{}, tmB{};
+  const void* A = nullptr;
+  const void* B = nullptr;
+  int K = 0;
+};
+
 }  // namespace
 
 // ============================================================== the handle
@@ -129,8 +161,11 @@ struct fd_handle {
   uint32_t magic = kMagic;
   fd_config cfg{};
   int bf = 0;                       // 1: bf16 storage + tcgen05 kernels
+  int paper = 0;                    // 1: the paper's output head
   int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
+  int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
+  size_t k_bytes = 0, v_bytes = 0, rk_bytes = 0, rv_bytes = 0;
   size_t latent_elems = 0, out_elems = 0, io_elt = 0, elt = 0;
 
   std::vector<void*> allocs;
@@ -141,8 +176,13 @@ struct fd_handle {
   std::vector<float*> bqkv, bo, b1, b2, gk, gv;
   void* wout = nullptr;
   float* bout = nullptr;
+  void *wup = nullptr, *wsp1 = nullptr;     // paper head
+  float *bup = nullptr, *bsp1 = nullptr;
   void *kc = nullptr, *vtc = nullptr;
+  void *rkc = nullptr, *rvtc = nullptr;     // refinement ring (paper head)
   float *x32 = nullptr, *ssq = nullptr;
+  float *xs32 = nullptr, *xss = nullptr;    // [r_t][L][D], [r_t][L][D/32]
+  void* xsb = nullptr;                      // [r_t][L][D] storage type
   void *xb = nullptr, *q = nullptr, *o = nullptr, *hb = nullptr;
   float2 *rope_row = nullptr, *rope_col = nullptr;
   long long* ctr = nullptr;
@@ -152,17 +192,17 @@ struct fd_handle {
 
   // TMA maps (bf16 path)
   CUtensorMap tm_xb{}, tm_o{}, tm_h{}, tm_q{}, tm_k{}, tm_v{}, tm_wout{};
-  std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_w1, tm_w2;
+  CUtensorMap tm_rk{}, tm_rv{}, tm_wup{}, tm_wsp1{}, tm_hs{};
+  std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_w1, tm_w2, tm_xs;
 
   // graph
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
   cudaGraphNode_t last_node = nullptr;
-  cudaGraphNode_t embed_node = nullptr, final_node = nullptr;
-  KernelLaunch embed_launch{}, final_launch{};
+  cudaGraphNode_t embed_node = nullptr;
+  KernelLaunch embed_launch{};
   EmbedParams embed_p{};
-  EpiParams final_p{};
-  int final_K = 0;
+  std::vector<OutNode> out_nodes;       // kernels writing the pixel buffer
   const void* cur_latent = nullptr;
   void* cur_out = nullptr;
   std::vector<cudaEvent_t> events;
@@ -264,7 +304,11 @@ struct fd_handle {
   fd_status_t add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, const void* A,
                        const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
                        cudaGraphNode_t* node);
-  EpiParams base_epi() const;
+  fd_status_t add_out_gemm(OutNode on, int N);
+  fd_status_t add_block(int wi, const BlockIO& io);
+  EpiParams base_epi(const BlockIO& io) const;
+  BlockIO backbone_io(int layer);
+  BlockIO subframe_io(int tau, int layer);
 };
 
 namespace {
@@ -301,32 +345,46 @@ const void* simt_gemm_fn(int dh) {
 
 }  // namespace
 
-EpiParams fd_handle::base_epi() const {
+EpiParams fd_handle::base_epi(const BlockIO& io) const {
   EpiParams e{};
   e.M = L;
-  e.ssq = ssq;
+  e.ssq = io.ssq;
   e.ssq_parts = cfg.d_model / 32;
   e.inv_d = 1.f / float(cfg.d_model);
   e.eps = cfg.norm_eps;
-  e.x32 = x32;
-  e.xb = xb;
-  e.ssq_out = ssq;
+  e.x32 = io.x32;
+  e.xb = io.xb;
+  e.ssq_out = io.ssq;
   e.D = cfg.d_model;
   e.q = q;
   e.H = cfg.n_heads;
   e.G = cfg.n_kv_heads;
   e.Dh = cfg.head_dim;
-  e.kv_rows = kv_rows;
-  e.vt_pitch = vt_pitch;
+  e.kv_rows = io.kv_rows;
+  e.vt_pitch = io.vt_pitch;
   e.kv_norm = cfg.kv_norm;
-  e.fs = fs;
+  e.fs = io.fs;
   e.rope_row = rope_row;
   e.rope_col = rope_col;
   e.tok_w = tok_w;
   e.tok_h = tok_h;
   e.P = cfg.px_per_token;
   e.out_bf16 = cfg.io_dtype == FD_BF16;
+  e.pl_mul = 1;
+  e.pl_add = 0;
   return e;
+}
+
+BlockIO fd_handle::backbone_io(int layer) {
+  return BlockIO{x32, xb, ssq, &tm_xb, kc, vtc, kv_rows, vt_pitch, &tm_k, &tm_v, layer, fs};
+}
+
+BlockIO fd_handle::subframe_io(int tau, int layer) {
+  const size_t rows = size_t(tau) * L;
+  const int D = cfg.d_model;
+  return BlockIO{xs32 + rows * D, static_cast<char*>(xsb) + rows * D * elt,
+                 xss + rows * (D / 32), bf ? &tm_xs[tau] : &tm_xb, rkc, rvtc, rkv_rows,
+                 rvt_pitch, &tm_rk, &tm_rv, layer, fs + 1 + tau};
 }
 
 // Kernel arguments must outlive the graph's construction; cudaGraphAddKernelNode
@@ -342,6 +400,7 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
       case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(L, N, num_sms, &bn, &k)); break;
       case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(L, N, num_sms, &bn, &k)); break;
       case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(L, N, num_sms, &bn, &k)); break;
+      case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(L, N, num_sms, &bn, &k)); break;
       default: FD_TRY(tc_gemm_pick<EPI_FINAL>(L, N, num_sms, &bn, &k)); break;
     }
     CUtensorMap a = tmA, b = tmB;
@@ -355,6 +414,7 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
     case EPI_QKV: k.func = simt_gemm_fn<EPI_QKV>(cfg.head_dim); break;
     case EPI_RESID: k.func = simt_gemm_fn<EPI_RESID>(cfg.head_dim); break;
     case EPI_GELU: k.func = simt_gemm_fn<EPI_GELU>(cfg.head_dim); break;
+    case EPI_UP: k.func = simt_gemm_fn<EPI_UP>(cfg.head_dim); break;
     default: k.func = simt_gemm_fn<EPI_FINAL>(cfg.head_dim); break;
   }
   k.grid = dim3((L + 127) / 128, N / 64);
@@ -368,6 +428,93 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
   return add_kernel(k, args, node);
 }
 
+// A FINAL GEMM whose output is the caller's pixel buffer; its launch and
+// arguments are kept so that fd_decode_frame can point it at a new buffer.
+fd_status_t fd_handle::add_out_gemm(OutNode on, int N) {
+  on.p.N = N;
+  FD_TRY(add_gemm(EPI_FINAL, FD_K_FINAL, on.tmA, on.A, on.tmB, on.B, N, on.K, on.p, &on.node));
+  cudaKernelNodeParams np{};
+  FD_CUDA(cudaGraphKernelNodeGetParams(on.node, &np));
+  on.launch = KernelLaunch{np.func, np.gridDim, np.blockDim, np.sharedMemBytes, FD_K_FINAL};
+  out_nodes.push_back(on);
+  return FD_OK;
+}
+
+// One Transformer block (weights wi) on the stream and cache of io
+// (paper Sec. 3.2-3.3): QKV (+RMSNorm, KV-norm, RoPE, ring write), window
+// attention, O-projection (+residual), MLP-up (+RMSNorm, GELU), MLP-down
+// (+residual).
+fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
+  const int D = cfg.d_model, H = cfg.n_heads, G = cfg.n_kv_heads, Dh = cfg.head_dim;
+  void* kc_l = static_cast<char*>(io.kc) + size_t(io.layer) * G * io.kv_rows * Dh * elt;
+  void* vtc_l = static_cast<char*>(io.vtc) + size_t(io.layer) * G * Dh * io.vt_pitch * elt;
+  // QKV + KV-norm + RoPE + ring write
+  EpiParams e = base_epi(io);
+  e.bias = bqkv[wi];
+  e.kc = kc_l;
+  e.vtc = vtc_l;
+  e.gk = gk[wi];
+  e.gv = gv[wi];
+  FD_TRY(add_gemm(EPI_QKV, FD_K_QKV, *io.tm_x, io.xb, bf ? tm_wqkv[wi] : *io.tm_x, wqkv[wi], qkv,
+                  D, e, nullptr));
+  // attention
+  if (bf) {
+    TcAttnParams ap{};
+    ap.o = o;
+    ap.L = L;
+    ap.H = H;
+    ap.G = G;
+    ap.layer = io.layer;
+    ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
+    ap.fs = io.fs;
+    ap.status = status;
+    // one 128-query tile per CTA, two CTAs per SM (measured faster than two
+    // query tiles sharing one CTA, and than three CTAs with single-buffered S)
+    using A = TcAttnSmem<1>;
+    const void* f = reinterpret_cast<const void*>(&tc_attn_kernel<1>);
+    FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
+    KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(A::kThreads), size_t(A::kAlloc), FD_K_ATTN};
+    CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;
+    void* args[] = {&a, &b, &c, &ap};
+    FD_TRY(add_kernel(k, args));
+  } else {
+    AttnParams ap{};
+    ap.q = q;
+    ap.kc = kc_l;
+    ap.vtc = vtc_l;
+    ap.o = o;
+    ap.L = L;
+    ap.H = H;
+    ap.G = G;
+    ap.kv_rows = io.kv_rows;
+    ap.vt_pitch = io.vt_pitch;
+    ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
+    ap.fs = io.fs;
+    ap.status = status;
+    const void* f = Dh == 32 ? reinterpret_cast<const void*>(&simt_attn_kernel<32>)
+                             : reinterpret_cast<const void*>(&simt_attn_kernel<64>);
+    KernelLaunch k{f, dim3((L + 63) / 64, H), dim3(64), 0, FD_K_ATTN};
+    void* args[] = {&ap};
+    FD_TRY(add_kernel(k, args));
+  }
+  // output projection + residual
+  e = base_epi(io);
+  e.bias = bo[wi];
+  FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[wi] : tm_o, wo[wi], D, H * Dh, e,
+                  nullptr));
+  // MLP up + GELU
+  e = base_epi(io);
+  e.bias = b1[wi];
+  e.hout = hb;
+  FD_TRY(add_gemm(EPI_GELU, FD_K_MLP_UP, *io.tm_x, io.xb, bf ? tm_w1[wi] : *io.tm_x, w1[wi], dff,
+                  D, e, nullptr));
+  // MLP down + residual
+  e = base_epi(io);
+  e.bias = b2[wi];
+  return add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h, hb, bf ? tm_w2[wi] : tm_h, w2[wi], D, dff, e,
+                  nullptr);
+}
+
 fd_status_t fd_handle::build_graph() {
   FD_CUDA(cudaGraphCreate(&graph, 0));
   last_node = nullptr;
@@ -379,9 +526,9 @@ fd_status_t fd_handle::build_graph() {
                    FD_K_STEP_BEGIN};
     long long* c = ctr;
     FrameState* f = fs;
-    int W = cfg.window, dh = cfg.head_dim;
+    int W = cfg.window, dh = cfg.head_dim, n_sub = paper ? cfg.r_t : 0;
     float th = cfg.rope_theta;
-    void* args[] = {&c, &f, &W, &dh, &th};
+    void* args[] = {&c, &f, &W, &dh, &th, &n_sub};
     FD_TRY(add_kernel(k, args));
   }
   // embed
@@ -409,88 +556,59 @@ fd_status_t fd_handle::build_graph() {
     FD_TRY(add_kernel(embed_launch, args, &embed_node));
     cur_latent = latent_stage;
   }
-  const int D = cfg.d_model, H = cfg.n_heads, Dh = cfg.head_dim;
-  for (int l = 0; l < cfg.n_blocks; ++l) {
-    // QKV + KV-norm + RoPE + ring write
-    EpiParams e = base_epi();
-    e.bias = bqkv[l];
-    e.kc = static_cast<char*>(kc) + size_t(l) * cfg.n_kv_heads * kv_rows * Dh * elt;
-    e.vtc = static_cast<char*>(vtc) + size_t(l) * cfg.n_kv_heads * Dh * vt_pitch * elt;
-    e.gk = gk[l];
-    e.gv = gv[l];
-    FD_TRY(add_gemm(EPI_QKV, FD_K_QKV, tm_xb, xb, bf ? tm_wqkv[l] : tm_xb, wqkv[l], qkv, D, e, nullptr));
-    // attention
-    if (bf) {
-      TcAttnParams ap{};
-      ap.o = o;
-      ap.L = L;
-      ap.H = H;
-      ap.G = cfg.n_kv_heads;
-      ap.layer = l;
-      ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
-      ap.fs = fs;
-      ap.status = status;
-      // one 128-query tile per CTA, two CTAs per SM (measured faster than two
-      // query tiles sharing one CTA, and than three CTAs with single-buffered S)
-      using A = TcAttnSmem<1>;
-      const void* f = reinterpret_cast<const void*>(&tc_attn_kernel<1>);
-      FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
-      KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(A::kThreads), size_t(A::kAlloc),
-                     FD_K_ATTN};
-      CUtensorMap a = tm_q, b = tm_k, c = tm_v;
-      void* args[] = {&a, &b, &c, &ap};
-      FD_TRY(add_kernel(k, args));
-    } else {
-      AttnParams ap{};
-      ap.q = q;
-      ap.kc = static_cast<char*>(kc) + size_t(l) * cfg.n_kv_heads * kv_rows * Dh * elt;
-      ap.vtc = static_cast<char*>(vtc) + size_t(l) * cfg.n_kv_heads * Dh * vt_pitch * elt;
-      ap.o = o;
-      ap.L = L;
-      ap.H = H;
-      ap.G = cfg.n_kv_heads;
-      ap.kv_rows = kv_rows;
-      ap.vt_pitch = vt_pitch;
-      ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
-      ap.fs = fs;
-      ap.status = status;
-      const void* f = Dh == 32 ? reinterpret_cast<const void*>(&simt_attn_kernel<32>)
-                               : reinterpret_cast<const void*>(&simt_attn_kernel<64>);
-      KernelLaunch k{f, dim3((L + 63) / 64, H), dim3(64), 0, FD_K_ATTN};
-      void* args[] = {&ap};
-      FD_TRY(add_kernel(k, args));
+  const int D = cfg.d_model;
+  for (int l = 0; l < cfg.n_blocks; ++l) FD_TRY(add_block(l, backbone_io(l)));
+
+  if (!paper) {
+    // final norm + projection + unpatchify
+    OutNode on;
+    on.p = base_epi(backbone_io(0));
+    on.p.bias = bout;
+    on.p.out = out_stage;
+    on.tmA = tm_xb;
+    on.A = xb;
+    on.tmB = bf ? tm_wout : tm_xb;
+    on.B = wout;
+    on.K = D;
+    FD_TRY(add_out_gemm(on, c_out));
+  } else {
+    // temporal upsampling (Eq. 3): xs[tau] = (up_w x + up_b)[tau D, (tau+1) D)
+    EpiParams e = base_epi(backbone_io(0));
+    e.bias = bup;
+    e.ssq = nullptr;
+    e.x32 = xs32;
+    e.xb = xsb;
+    e.ssq_out = xss;
+    FD_TRY(add_gemm(EPI_UP, FD_K_UPSAMPLE, tm_xb, xb, bf ? tm_wup : tm_xb, wup, cfg.r_t * D, D, e,
+                    nullptr));
+    const int c_px = cfg.out_ch * cfg.px_per_token * cfg.px_per_token;
+    for (int tau = 0; tau < cfg.r_t; ++tau) {
+      // refinement blocks: sub-frame t r_t + tau in the ring of r_t (W+1)
+      for (int l = 0; l < cfg.n_refine; ++l) FD_TRY(add_block(cfg.n_blocks + l, subframe_io(tau, l)));
+      // spatial MLP layer 1: GELU(RMSNorm(xs) sp1_w^T + sp1_b) -> hidden [L][D]
+      const BlockIO io = subframe_io(tau, 0);
+      e = base_epi(io);
+      e.bias = bsp1;
+      e.hout = hb;
+      FD_TRY(add_gemm(EPI_GELU, FD_K_SPATIAL, *io.tm_x, io.xb, bf ? tm_wsp1 : *io.tm_x, wsp1, D,
+                      D, e, nullptr));
+      // layer 2 + PixelShuffle into pixel frames (c, tau), no norm
+      OutNode on;
+      on.p = base_epi(io);
+      on.p.bias = bout;
+      on.p.ssq = nullptr;
+      on.p.out = out_stage;
+      on.p.pl_mul = cfg.r_t;
+      on.p.pl_add = tau;
+      on.tmA = bf ? tm_hs : tm_xb;
+      on.A = hb;
+      on.tmB = bf ? tm_wout : tm_xb;
+      on.B = wout;
+      on.K = D;
+      FD_TRY(add_out_gemm(on, c_px));
     }
-    // output projection + residual
-    e = base_epi();
-    e.bias = bo[l];
-    FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[l] : tm_o, wo[l], D, H * Dh, e,
-                    nullptr));
-    // MLP up + GELU
-    e = base_epi();
-    e.bias = b1[l];
-    e.hout = hb;
-    FD_TRY(add_gemm(EPI_GELU, FD_K_MLP_UP, tm_xb, xb, bf ? tm_w1[l] : tm_xb, w1[l], dff, D, e,
-                    nullptr));
-    // MLP down + residual
-    e = base_epi();
-    e.bias = b2[l];
-    FD_TRY(add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h, hb, bf ? tm_w2[l] : tm_h, w2[l], D, dff, e,
-                    nullptr));
   }
-  // final norm + projection + unpatchify
-  {
-    final_p = base_epi();
-    final_p.bias = bout;
-    final_p.out = out_stage;
-    final_K = D;
-    FD_TRY(add_gemm(EPI_FINAL, FD_K_FINAL, tm_xb, xb, bf ? tm_wout : tm_xb, wout, c_out, D,
-                    final_p, &final_node));
-    final_p.N = c_out;
-    cudaKernelNodeParams np{};
-    FD_CUDA(cudaGraphKernelNodeGetParams(final_node, &np));
-    final_launch = KernelLaunch{np.func, np.gridDim, np.blockDim, np.sharedMemBytes, FD_K_FINAL};
-    cur_out = out_stage;
-  }
+  cur_out = out_stage;
   FD_CUDA(cudaGraphInstantiate(&exec, graph, 0));
   return FD_OK;
 }
@@ -541,6 +659,17 @@ fd_status_t validate(const fd_config* c) {
                 L * (c->window + 1));
   if (c->kernel_timing < 0 || c->kernel_timing > 2)
     return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0, 1 or 2");
+  if (c->head_mode != 0 && c->head_mode != 1)
+    return fail(FD_ERR_INVALID_ARG, "config: head_mode must be 0 or 1");
+  if (c->head_mode == 1) {
+    if (c->n_refine < 1 || c->n_refine > 8)
+      return fail(FD_ERR_UNSUPPORTED, "config: n_refine must be 1 .. 8 (got %d)", c->n_refine);
+    if (c->r_t > 16)
+      return fail(FD_ERR_UNSUPPORTED, "config: the paper head supports r_t <= 16 (got %d)", c->r_t);
+    if (L * c->r_t * (c->window + 1) > (1LL << 30))
+      return fail(FD_ERR_UNSUPPORTED, "config: refinement window of %lld tokens is too large",
+                  L * c->r_t * (c->window + 1));
+  }
   return FD_OK;
 }
 
@@ -548,6 +677,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   h->cfg = *cfg;
   const fd_config& c = *cfg;
   h->bf = c.dtype == FD_BF16;
+  h->paper = c.head_mode == 1;
   h->elt = h->bf ? 2 : 4;
   h->io_elt = c.io_dtype == FD_BF16 ? 2 : 4;
   h->tok_h = c.grid_h / c.patch;
@@ -559,6 +689,8 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   h->c_out = c.out_ch * c.r_t * c.px_per_token * c.px_per_token;
   h->kv_rows = (c.window + 1) * h->L;
   h->vt_pitch = int(round_up(size_t(h->kv_rows), 64));
+  h->rkv_rows = c.r_t * (c.window + 1) * h->L;
+  h->rvt_pitch = int(round_up(size_t(h->rkv_rows), 64));
   h->out_h = h->tok_h * c.px_per_token;
   h->out_w = h->tok_w * c.px_per_token;
   h->latent_elems = size_t(c.latent_ch) * c.grid_h * c.grid_w;
@@ -573,6 +705,8 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
                 major);
 
   const int D = c.d_model, H = c.n_heads, G = c.n_kv_heads, Dh = c.head_dim, NB = c.n_blocks;
+  const int NR = h->paper ? c.n_refine : 0;        // refinement blocks follow the backbone's
+  const int c_px = c.out_ch * c.px_per_token * c.px_per_token;
   // ---- weights
   {
     std::vector<float> wT(size_t(h->c_in) * D);
@@ -582,7 +716,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(h->upload_f32(&h->embed_b, w->embed_b, D));
   }
   std::vector<float> ones(std::max(D, Dh), 1.f);
-  for (int l = 0; l < NB; ++l) {
+  for (int l = 0; l < NB + NR; ++l) {
     void* p;
     FD_TRY(h->upload_w(&p, w->wqkv[l], h->qkv, D, w->norm1_g[l])); h->wqkv.push_back(p);
     FD_TRY(h->upload_w(&p, w->wo[l], D, size_t(H) * Dh, nullptr)); h->wo.push_back(p);
@@ -596,15 +730,32 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(h->upload_f32(&f, c.kv_norm ? w->knorm_g[l] : ones.data(), Dh)); h->gk.push_back(f);
     FD_TRY(h->upload_f32(&f, c.kv_norm ? w->vnorm_g[l] : ones.data(), Dh)); h->gv.push_back(f);
   }
-  FD_TRY(h->upload_w(&h->wout, w->out_w, h->c_out, D, w->final_g));
-  FD_TRY(h->upload_f32(&h->bout, w->out_b, h->c_out));
+  if (!h->paper) {
+    FD_TRY(h->upload_w(&h->wout, w->out_w, h->c_out, D, w->final_g));
+    FD_TRY(h->upload_f32(&h->bout, w->out_b, h->c_out));
+  } else {
+    // final_g is the RMSNorm before the spatial MLP: folded into its first layer
+    FD_TRY(h->upload_w(&h->wup, w->up_w, size_t(c.r_t) * D, D, nullptr));
+    FD_TRY(h->upload_f32(&h->bup, w->up_b, size_t(c.r_t) * D));
+    FD_TRY(h->upload_w(&h->wsp1, w->sp1_w, D, D, w->final_g));
+    FD_TRY(h->upload_f32(&h->bsp1, w->sp1_b, D));
+    FD_TRY(h->upload_w(&h->wout, w->out_w, c_px, D, nullptr));
+    FD_TRY(h->upload_f32(&h->bout, w->out_b, c_px));
+  }
 
-  // ---- ring cache: K [NB][G][(W+1)L][Dh], V^T [NB][G][Dh][vt_pitch]
-  const size_t k_bytes = size_t(NB) * G * h->kv_rows * Dh * h->elt;
-  const size_t v_bytes = size_t(NB) * G * Dh * h->vt_pitch * h->elt;
-  FD_TRY(h->alloc(&h->kc, k_bytes));
-  FD_TRY(h->alloc(&h->vtc, v_bytes));
-  h->cache_bytes = k_bytes + v_bytes;
+  // ---- ring caches: K [layers][G][rows][Dh], V^T [layers][G][Dh][pitch];
+  // backbone rows = (W+1) L, refinement rows = r_t (W+1) L
+  h->k_bytes = size_t(NB) * G * h->kv_rows * Dh * h->elt;
+  h->v_bytes = size_t(NB) * G * Dh * h->vt_pitch * h->elt;
+  FD_TRY(h->alloc(&h->kc, h->k_bytes));
+  FD_TRY(h->alloc(&h->vtc, h->v_bytes));
+  if (h->paper) {
+    h->rk_bytes = size_t(NR) * G * h->rkv_rows * Dh * h->elt;
+    h->rv_bytes = size_t(NR) * G * Dh * h->rvt_pitch * h->elt;
+    FD_TRY(h->alloc(&h->rkc, h->rk_bytes));
+    FD_TRY(h->alloc(&h->rvtc, h->rv_bytes));
+  }
+  h->cache_bytes = h->k_bytes + h->v_bytes + h->rk_bytes + h->rv_bytes;
 
   // ---- scratch
   const size_t L = h->L;
@@ -614,8 +765,13 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   FD_TRY(h->alloc(&h->q, size_t(H) * L * Dh * h->elt));
   FD_TRY(h->alloc(&h->o, L * H * Dh * h->elt));
   FD_TRY(h->alloc(&h->hb, L * h->dff * h->elt));
+  if (h->paper) {
+    FD_TRY(h->alloc(&h->xs32, size_t(c.r_t) * L * D * 4));
+    FD_TRY(h->alloc(&h->xsb, size_t(c.r_t) * L * D * h->elt));
+    FD_TRY(h->alloc(&h->xss, size_t(c.r_t) * L * (D / 32) * 4));
+  }
   FD_TRY(h->alloc(&h->ctr, 64));
-  FD_TRY(h->alloc(&h->fs, sizeof(FrameState)));
+  FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * (1 + (h->paper ? c.r_t : 0))));
   FD_TRY(h->alloc(&h->status, 16));
   FD_TRY(h->alloc(&h->latent_stage, round_up(h->latent_elems * h->io_elt, 256)));
   FD_TRY(h->alloc(&h->out_stage, round_up(h->out_elems * h->io_elt, 256)));
@@ -646,14 +802,33 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(make_tmap_2d(&h->tm_o, h->o, L, size_t(H) * Dh, 128));
     FD_TRY(make_tmap_2d(&h->tm_h, h->hb, L, h->dff, 128));
     auto bn_of = [](int N) { return N % 256 == 0 ? 256u : (N % 128 == 0 ? 128u : 64u); };
-    for (int l = 0; l < NB; ++l) {
+    for (int l = 0; l < NB + NR; ++l) {
       CUtensorMap m;
       FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(h->qkv))); h->tm_wqkv.push_back(m);
       FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D))); h->tm_wo.push_back(m);
       FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
       FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
     }
-    FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, h->c_out, D, bn_of(h->c_out)));
+    const int n_out = h->paper ? c_px : h->c_out;
+    FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, n_out, D, bn_of(n_out)));
+    if (h->paper) {
+      FD_TRY(make_tmap_2d(&h->tm_wup, h->wup, size_t(c.r_t) * D, D, bn_of(c.r_t * D)));
+      FD_TRY(make_tmap_2d(&h->tm_wsp1, h->wsp1, D, D, bn_of(D)));
+      FD_TRY(make_tmap_2d(&h->tm_hs, h->hb, L, D, 128));          // spatial hidden [L][D]
+      for (int tau = 0; tau < c.r_t; ++tau) {
+        CUtensorMap m;
+        FD_TRY(make_tmap_2d(&m, static_cast<char*>(h->xsb) + size_t(tau) * L * D * 2, L, D, 128));
+        h->tm_xs.push_back(m);
+      }
+      const uint64_t kd[3] = {64, uint64_t(h->rkv_rows), uint64_t(NR) * G};
+      const uint64_t ks[2] = {64 * 2, uint64_t(h->rkv_rows) * 64 * 2};
+      const uint32_t kb[3] = {64, 64, 1};
+      FD_TRY(make_tmap(&h->tm_rk, h->rkc, 3, kd, ks, kb));
+      const uint64_t vd[3] = {uint64_t(h->rvt_pitch), 64, uint64_t(NR) * G};
+      const uint64_t vs[2] = {uint64_t(h->rvt_pitch) * 2, uint64_t(h->rvt_pitch) * 64 * 2};
+      const uint32_t vb[3] = {64, 64, 1};
+      FD_TRY(make_tmap(&h->tm_rv, h->rvtc, 3, vd, vs, vb));
+    }
     {   // Q [H][L][64]: box 64 x 128 x 1
       const uint64_t dims[3] = {64, L, uint64_t(H)};
       const uint64_t str[2] = {64 * 2, L * 64 * 2};
@@ -675,8 +850,12 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   }
 
   // ---- reset state, build the graph
-  FD_CUDA(cudaMemset(h->kc, 0, k_bytes));
-  FD_CUDA(cudaMemset(h->vtc, 0, v_bytes));
+  FD_CUDA(cudaMemset(h->kc, 0, h->k_bytes));
+  FD_CUDA(cudaMemset(h->vtc, 0, h->v_bytes));
+  if (h->paper) {
+    FD_CUDA(cudaMemset(h->rkc, 0, h->rk_bytes));
+    FD_CUDA(cudaMemset(h->rvtc, 0, h->rv_bytes));
+  }
   FD_CUDA(cudaMemset(h->ctr, 0, 64));
   FD_CUDA(cudaMemset(h->status, 0, 16));
   FD_CUDA(cudaMemset(h->fs, 0, sizeof(FrameState)));
@@ -699,26 +878,27 @@ fd_status_t patch_io(fd_handle* h, const void* latent, void* out) {
     h->cur_latent = latent;
   }
   if (out != h->cur_out) {
-    h->final_p.out = out;
-    cudaKernelNodeParams np{};
-    np.func = const_cast<void*>(h->final_launch.func);
-    np.gridDim = h->final_launch.grid;
-    np.blockDim = h->final_launch.block;
-    np.sharedMemBytes = unsigned(h->final_launch.smem);
-    if (h->bf) {
-      CUtensorMap a = h->tm_xb, b = h->tm_wout;
-      int K = h->final_K;
-      int* st = h->status;
-      void* args[] = {&a, &b, &K, &h->final_p, &st};
-      np.kernelParams = args;
-      FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, h->final_node, &np));
-    } else {
-      const float* a = static_cast<const float*>(h->xb);
-      const float* b = static_cast<const float*>(h->wout);
-      int K = h->final_K;
-      void* args[] = {&a, &b, &K, &h->final_p};
-      np.kernelParams = args;
-      FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, h->final_node, &np));
+    for (OutNode& on : h->out_nodes) {
+      on.p.out = out;
+      cudaKernelNodeParams np{};
+      np.func = const_cast<void*>(on.launch.func);
+      np.gridDim = on.launch.grid;
+      np.blockDim = on.launch.block;
+      np.sharedMemBytes = unsigned(on.launch.smem);
+      int K = on.K;
+      if (h->bf) {
+        CUtensorMap a = on.tmA, b = on.tmB;
+        int* st = h->status;
+        void* args[] = {&a, &b, &K, &on.p, &st};
+        np.kernelParams = args;
+        FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, on.node, &np));
+      } else {
+        const float* a = static_cast<const float*>(on.A);
+        const float* b = static_cast<const float*>(on.B);
+        void* args[] = {&a, &b, &K, &on.p};
+        np.kernelParams = args;
+        FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, on.node, &np));
+      }
     }
     h->cur_out = out;
   }
@@ -737,9 +917,11 @@ fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle
   const fd_weights* w = weights;
   if (!w->embed_w || !w->embed_b || !w->norm1_g || !w->wqkv || !w->bqkv || !w->wo || !w->bo ||
       !w->norm2_g || !w->w1 || !w->b1 || !w->w2 || !w->b2 || !w->final_g || !w->out_w ||
-      !w->out_b || (cfg->kv_norm && (!w->knorm_g || !w->vnorm_g)))
+      !w->out_b || (cfg->kv_norm && (!w->knorm_g || !w->vnorm_g)) ||
+      (cfg->head_mode == 1 && (!w->up_w || !w->up_b || !w->sp1_w || !w->sp1_b)))
     return fail(FD_ERR_INVALID_ARG, "fd_create: null weight pointer");
-  for (int l = 0; l < cfg->n_blocks; ++l)
+  const int n_all = cfg->n_blocks + (cfg->head_mode == 1 ? cfg->n_refine : 0);
+  for (int l = 0; l < n_all; ++l)
     if (!w->norm1_g[l] || !w->wqkv[l] || !w->bqkv[l] || !w->wo[l] || !w->bo[l] ||
         !w->norm2_g[l] || !w->w1[l] || !w->b1[l] || !w->w2[l] || !w->b2[l] ||
         (cfg->kv_norm && (!w->knorm_g[l] || !w->vnorm_g[l])))
@@ -760,10 +942,12 @@ fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle
 fd_status_t fd_reset(fd_handle* h, void* stream) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_reset: invalid handle");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  FD_CUDA(cudaMemsetAsync(h->kc, 0, size_t(h->cfg.n_blocks) * h->cfg.n_kv_heads * h->kv_rows *
-                                        h->cfg.head_dim * h->elt, s));
-  FD_CUDA(cudaMemsetAsync(h->vtc, 0, size_t(h->cfg.n_blocks) * h->cfg.n_kv_heads *
-                                         h->cfg.head_dim * h->vt_pitch * h->elt, s));
+  FD_CUDA(cudaMemsetAsync(h->kc, 0, h->k_bytes, s));
+  FD_CUDA(cudaMemsetAsync(h->vtc, 0, h->v_bytes, s));
+  if (h->paper) {
+    FD_CUDA(cudaMemsetAsync(h->rkc, 0, h->rk_bytes, s));
+    FD_CUDA(cudaMemsetAsync(h->rvtc, 0, h->rv_bytes, s));
+  }
   FD_CUDA(cudaMemsetAsync(h->ctr, 0, 64, s));
   FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
   h->last_stream = s;

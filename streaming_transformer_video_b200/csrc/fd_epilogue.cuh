@@ -8,8 +8,11 @@
 //   RESID  residual add into the fp32 stream x, its storage-type copy and
 //          the per-32-column sums of squares the next RMSNorm needs
 //   GELU   RMSNorm row scale + bias + exact GELU -> MLP hidden
-//   FINAL  RMSNorm row scale + bias -> unpatchify scatter into NCTHW pixels
+//   FINAL  [RMSNorm row scale] + bias -> unpatchify scatter into NCTHW pixels
 //          (Sec. 3.4, Step 3: depth-to-space)
+//   UP     bias -> temporal upsampling (Sec. 3.4, Eq. 3): output channels
+//          [tau D, (tau+1) D) become the residual stream of sub-frame tau
+//          (fp32 copy, storage-type copy, per-32-column sums of squares)
 //
 // RMSNorm fusion: the gain g is folded into the following weight matrix at
 // create time, so RMSNorm(x) W^T = diag(r) (x (W diag g)^T) with
@@ -21,18 +24,24 @@
 
 namespace fd {
 
-enum EpiKind { EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2, EPI_FINAL = 3 };
+enum EpiKind { EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2, EPI_FINAL = 3, EPI_UP = 4 };
+
+// Kinds whose A operand is an RMSNorm input (their rows get the row scale);
+// a null EpiParams::ssq turns the scale off (the spatial MLP's second layer).
+constexpr bool epi_normed(int kind) {
+  return kind == EPI_QKV || kind == EPI_GELU || kind == EPI_FINAL;
+}
 
 struct EpiParams {
   int M;                 // rows (tokens of the frame)
   int N;                 // GEMM output columns
   const float* bias;     // [N]
-  // RMSNorm row scale (QKV, GELU, FINAL)
+  // RMSNorm row scale (QKV, GELU, FINAL; none when ssq is null)
   const float* ssq;      // [M][ssq_parts] sums of squares of x
   int ssq_parts;
   float inv_d;           // 1 / D
   float eps;
-  // RESID
+  // RESID (UP: the same three buffers with a leading sub-frame index)
   float* x32;            // [M][D] fp32 residual stream (updated in place)
   void* xb;              // [M][D] storage-type copy (next GEMM's A operand)
   float* ssq_out;        // [M][D/32]
@@ -58,6 +67,8 @@ struct EpiParams {
   int out_bf16;          // pixel element type
   int P;                 // pixels per token side
   int tok_h;
+  int pl_mul, pl_add;    // column block c = col / P^2 goes to pixel frame
+                         // c * pl_mul + pl_add of the [C * r_t] output frames
 };
 
 __device__ __forceinline__ float row_scale(const EpiParams& p, int row) {
@@ -181,6 +192,24 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
 #pragma unroll
     for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * rs + __ldg(p.bias + col0 + c));
     store_vec<T, 64>(static_cast<T*>(p.hout) + size_t(row) * p.N + col0, acc);
+  } else if constexpr (KIND == EPI_UP) {
+    const int tau = col0 / p.D, c0 = col0 - tau * p.D;
+    const size_t r = size_t(tau) * p.M + row;             // row of sub-frame tau
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] += __ldg(p.bias + col0 + c);
+    float* x = p.x32 + r * p.D + c0;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4)
+      *reinterpret_cast<float4*>(x + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+    store_vec<T, 64>(static_cast<T*>(p.xb) + r * p.D + c0, acc);
+    const int parts = p.D / 32;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) s += acc[h * 32 + c] * acc[h * 32 + c];
+      p.ssq_out[r * parts + c0 / 32 + h] = s;
+    }
   } else {  // EPI_FINAL
 #pragma unroll
     for (int c = 0; c < 64; ++c) acc[c] = acc[c] * rs + __ldg(p.bias + col0 + c);
@@ -188,11 +217,13 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
     const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
     const size_t out_w = size_t(p.tok_w) * P;
     const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
-    // 64 columns = 64/P output rows of P pixels each; column
-    // ((c*r_t + tau)*P + dy)*P + dx maps to frame (c, tau), pixel row i*P+dy.
+    // 64 columns = 64/P output rows of P pixels each; column (b*P + dy)*P + dx
+    // maps to pixel frame b*pl_mul + pl_add, pixel row i*P+dy. The linear head
+    // has b = c*r_t + tau (pl_mul 1, pl_add 0); the spatial MLP of sub-frame
+    // tau has b = c (pl_mul r_t, pl_add tau).
     for (int s = 0; s < 64; s += P) {
       const int col = col0 + s;
-      const int ct = col / (P * P);                 // c*r_t + tau
+      const int ct = (col / (P * P)) * p.pl_mul + p.pl_add;
       const int dy = (col / P) % P;
       const size_t off = size_t(ct) * plane + (size_t(i) * P + dy) * out_w + size_t(j) * P;
       if (p.out_bf16) {

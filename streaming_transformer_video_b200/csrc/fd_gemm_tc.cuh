@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int row = m_blk * 128 + quarter * 32 + lane;
       float rs = 1.f;
-      if (KIND != EPI_RESID && row < M) rs = row_scale(ep, row);
+      if (epi_normed(KIND) && row < M && ep.ssq) rs = row_scale(ep, row);
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + buf * BN;
 #pragma unroll 1
       for (int c = 64 * half; c < BN; c += 64 * kPerQuarter) {

@@ -14,16 +14,14 @@
 namespace fd {
 
 // ---------------------------------------------------------------- step_begin
-// t = counter; slot = t mod (W+1); n_valid = min(t, W) + 1; temporal RoPE
+// Frame state of one streamed frame with absolute index t in a ring of `cap`
+// slots: slot = t mod cap; n_valid = min(t, cap - 1) + 1; temporal RoPE
 // angles t * theta^(-2m/d_t) reduced mod 2 pi in fp64 so they stay exact for
-// any stream length; counter = t + 1.
-__global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int head_dim,
-                                  float theta) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  const long long t = *ctr;
+// any stream length.
+__device__ void frame_state(FrameState* fs, long long t, int cap, int head_dim, float theta) {
   fs->t = t;
-  fs->slot = int(t % (W + 1));
-  fs->n_valid = int(t < W ? t : W) + 1;
+  fs->slot = int(t % cap);
+  fs->n_valid = int(t < cap - 1 ? t : cap - 1) + 1;
   const int dt = head_dim / 4;
   const double two_pi = 6.283185307179586476925286766559;
   for (int m = 0; m < dt / 2; ++m) {
@@ -31,7 +29,24 @@ __global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int hea
     const double ang = fmod(double(t) * freq, two_pi);
     fs->rope_t[m] = make_float2(float(cos(ang)), float(sin(ang)));
   }
-  *ctr = t + 1;
+}
+
+// fs[0]: latent frame t = counter in the backbone ring of W+1 frames.
+// fs[1 + tau], tau < n_sub (paper head, n_sub = r_t): sub-frame t r_t + tau
+// in the refinement ring of r_t (W+1) sub-frames (paper Sec. 3.4, Step 2).
+// Thread tau + 1 writes sub-frame tau; the counter becomes t + 1.
+__global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int head_dim,
+                                  float theta, int n_sub) {
+  if (blockIdx.x != 0) return;
+  const long long t = *ctr;
+  __syncwarp();
+  const int i = threadIdx.x;
+  if (i == 0) {
+    frame_state(fs, t, W + 1, head_dim, theta);
+    *ctr = t + 1;
+  } else if (i <= n_sub) {
+    frame_state(fs + i, t * n_sub + (i - 1), n_sub * (W + 1), head_dim, theta);
+  }
 }
 
 // ---------------------------------------------------------------- self-test
@@ -143,7 +158,7 @@ __global__ void __launch_bounds__(128) simt_gemm_kernel(const float* A, const fl
     __syncthreads();
   }
   if (row < p.M) {
-    const float rs = (KIND == EPI_RESID) ? 1.f : row_scale(p, row);
+    const float rs = (epi_normed(KIND) && p.ssq) ? row_scale(p, row) : 1.f;
     epilogue64<KIND, float, DH>(p, row, col0, acc, rs);
   }
 }

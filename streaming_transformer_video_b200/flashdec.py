@@ -20,7 +20,9 @@ LIB_PATH = os.path.join(_HERE, "libflashdec.so")
 FD_OK, FD_ERR_INVALID_ARG, FD_ERR_UNSUPPORTED, FD_ERR_OOM = 0, -1, -2, -3
 FD_ERR_CUDA, FD_ERR_TIMEOUT, FD_ERR_BAD_HANDLE = -4, -5, -6
 FD_F32, FD_BF16 = 0, 1
-KERNEL_KINDS = ["step_begin", "embed", "qkv", "attn", "oproj", "mlp_up", "mlp_down", "final"]
+KERNEL_KINDS = ["step_begin", "embed", "qkv", "attn", "oproj", "mlp_up", "mlp_down", "final",
+                "upsample", "spatial"]
+HEAD_MODES = {"linear": 0, "paper": 1}
 
 EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
@@ -34,7 +36,8 @@ class FDConfigC(ctypes.Structure):
         "head_dim", "n_blocks", "mlp_ratio", "window", "out_ch", "r_t", "px_per_token",
         "kv_norm", "dtype", "io_dtype")] + [
         ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
-        ("kernel_timing", ctypes.c_int32)]
+        ("kernel_timing", ctypes.c_int32), ("head_mode", ctypes.c_int32),
+        ("n_refine", ctypes.c_int32)]
 
 
 _PF = ctypes.POINTER(ctypes.c_float)
@@ -47,7 +50,8 @@ class FDWeightsC(ctypes.Structure):
                 ("knorm_g", _PPF), ("vnorm_g", _PPF),
                 ("wo", _PPF), ("bo", _PPF), ("norm2_g", _PPF),
                 ("w1", _PPF), ("b1", _PPF), ("w2", _PPF), ("b2", _PPF),
-                ("final_g", _PF), ("out_w", _PF), ("out_b", _PF)]
+                ("final_g", _PF), ("out_w", _PF), ("out_b", _PF),
+                ("up_w", _PF), ("up_b", _PF), ("sp1_w", _PF), ("sp1_b", _PF)]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -131,6 +135,8 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
     c.rope_theta = float(getattr(cfg, "rope_theta", 1e4))
     # False/0: off; True/1: every kernel; 2: attention launches only
     c.kernel_timing = int(kernel_timing)
+    c.head_mode = HEAD_MODES[getattr(cfg, "head", "linear")]
+    c.n_refine = int(getattr(cfg, "n_refine", 0)) if c.head_mode else 0
     return c
 
 
@@ -150,6 +156,8 @@ class FlashDecoder:
     "embed_w", "embed_b", "b{l}.norm1_g", "b{l}.wqkv", "b{l}.bqkv",
     "b{l}.knorm_g", "b{l}.vnorm_g", "b{l}.wo", "b{l}.bo", "b{l}.norm2_g",
     "b{l}.w1", "b{l}.b1", "b{l}.w2", "b{l}.b2", "final_g", "out_w", "out_b".
+    With cfg.head == "paper" also "up_w", "up_b", "sp1_w", "sp1_b" and the
+    refinement blocks "r{l}.*" (same keys as "b{l}.*"), l < cfg.n_refine.
     """
 
     def __init__(self, cfg, weights: Dict[str, np.ndarray], io_dtype=None,
@@ -164,8 +172,12 @@ class FlashDecoder:
             keep.append(a)
             return a.ctypes.data_as(_PF)
 
+        prefixes = [f"b{l}." for l in range(cfg.n_blocks)]
+        if self.c.head_mode:
+            prefixes += [f"r{l}." for l in range(cfg.n_refine)]
+
         def per_block(key):
-            arr = (_PF * cfg.n_blocks)(*[fp(f"b{l}.{key}") for l in range(cfg.n_blocks)])
+            arr = (_PF * len(prefixes))(*[fp(p + key) for p in prefixes])
             keep.append(arr)
             return ctypes.cast(arr, _PPF)
 
@@ -175,6 +187,9 @@ class FlashDecoder:
                     "w1", "b1", "w2", "b2"):
             setattr(w, key, per_block(key))
         w.final_g, w.out_w, w.out_b = fp("final_g"), fp("out_w"), fp("out_b")
+        if self.c.head_mode:
+            w.up_w, w.up_b, w.sp1_w, w.sp1_b = (fp("up_w"), fp("up_b"), fp("sp1_w"),
+                                                fp("sp1_b"))
         h = ctypes.c_void_p()
         _check(self._lib.fd_create(ctypes.byref(self.c), ctypes.byref(w), ctypes.byref(h)),
                "fd_create")

@@ -93,6 +93,16 @@ def test_create_rejects_bad_configs_before_touching_the_device():
         s, _ = _create(c)
         assert s == code, (kw, s, lib.fd_last_error())
         assert lib.fd_last_error().decode()
+    # output head fields (set on the C struct directly)
+    paper = base.replace(head="paper")
+    for field, value, code in [("head_mode", 2, fdb.FD_ERR_INVALID_ARG),
+                               ("n_refine", 0, fdb.FD_ERR_UNSUPPORTED),
+                               ("n_refine", 9, fdb.FD_ERR_UNSUPPORTED),
+                               ("r_t", 17, fdb.FD_ERR_UNSUPPORTED)]:
+        c = fdb.make_config(paper)
+        setattr(c, field, value)
+        s, _ = _create(c)
+        assert s == code, (field, value, s, lib.fd_last_error())
     # valid shape but null weights
     s, _ = _create(fdb.make_config(base))
     assert s == fdb.FD_ERR_INVALID_ARG
