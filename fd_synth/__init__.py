@@ -60,6 +60,9 @@ class FDConfig:
     # PixelShuffle per sub-frame (paper Sec. 3.4)
     head: str = "linear"
     n_refine: int = 2
+    # 1: the MLP sublayer of every Transformer block runs on FP8 E4M3 operands
+    # with static per-tensor scales (paper Sec. 4.6); bf16 configurations only
+    mlp_fp8: int = 0
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property

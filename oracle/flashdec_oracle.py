@@ -28,6 +28,17 @@ notes of the repository):
     layers carry biases.
   * Output head: RMSNorm, one Linear D -> C*r_t*P^2 with channel order
     (c, tau, dy, dx), then unpatchify to [C][r_t][H_tok*P][W_tok*P].
+  * FP8 MLP ([FD] Sec. 4.6, "static-calibrated FP8 quantization of all MLP
+    layers"): the MLP sublayer of every Transformer block (backbone and
+    refinement; not the pixel head's spatial MLP) multiplies E4M3 operands.
+    Per-tensor static scales: each weight matrix s_w = max|W| / 448; the
+    activations entering each Linear have a scale fixed by calibration
+    (max |activation| over calibration frames / 448). The first Linear's
+    operand is the residual stream x itself: the RMSNorm gain is folded into
+    W_1 before W_1 is quantized and the RMSNorm row scale multiplies the
+    product, so only the point where the rounding happens differs from
+    quantizing the normalised input. The hidden activation is quantized
+    after GELU. Rounding: nearest, ties to even, saturating at +-448.
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py
 (library routines, closed forms, invariants of the method). No function
@@ -90,6 +101,80 @@ def rms_norm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
 def gelu(x: np.ndarray) -> np.ndarray:
     """Exact GELU: x * Phi(x) = x/2 (1 + erf(x/sqrt 2))."""
     return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 quantization of the MLP layers ([FD] Sec. 4.6, optimization (4))
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0          # largest finite E4M3 value: 1.75 * 2^8
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Nearest value of the FP8 E4M3 format: 1 sign bit, 4 exponent bits
+    with bias 7, 3 fraction bits, no infinities (normal numbers
+    (1 + f/8) 2^(e-7), e = 1..15, except e = 15, f = 7, which encodes NaN;
+    subnormals (f/8) 2^-6). Ties go to the even neighbour; finite values and
+    infinities beyond +-448 saturate to +-448; NaN stays NaN. Returns the
+    rounded values as float64."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)                     # a = m 2^ex, m in [0.5, 1)
+    e = np.maximum(ex - 1, -6)              # binade 2^e; below 2^-6 the subnormal spacing
+    step = np.ldexp(1.0, e - 3)             # 3 fraction bits
+    with np.errstate(invalid="ignore"):
+        q = np.minimum(np.round(a / step) * step, E4M3_MAX)   # np.round: ties to even
+    return np.where(np.isnan(v), np.nan, np.copysign(q, v))
+
+
+def weight_scale(w: np.ndarray) -> float:
+    """Static per-tensor scale of a weight matrix: fp32(max|w| / 448), or 1
+    for an all-zero matrix."""
+    amax = float(np.max(np.abs(w)))
+    return float(np.float32(amax / E4M3_MAX)) if amax > 0 else 1.0
+
+
+def quantize_weight(w: np.ndarray, s: float) -> np.ndarray:
+    """Dequantized FP8 weight e4m3(w / s) s (division in float64)."""
+    return e4m3_round(np.asarray(w, dtype=np.float64) / np.float64(s)) * np.float64(s)
+
+
+def quantize_act(x: np.ndarray, s: float) -> np.ndarray:
+    """Dequantized FP8 activation with static scale s: e4m3(x * (1/s)) s,
+    where x, 1/s and their product are float32 (the precision in which the
+    device takes the same rounding decision)."""
+    inv = np.float32(1.0 / np.float64(s))
+    v = np.asarray(x, dtype=np.float64).astype(np.float32) * inv
+    return e4m3_round(v.astype(np.float64)) * np.float64(s)
+
+
+def mlp(cfg, w: Dict[str, np.ndarray], p: str, x: np.ndarray,
+        amax: Optional[Dict[str, float]] = None) -> np.ndarray:
+    """Pre-norm MLP sublayer of block p (without the residual add):
+    GELU(RMSNorm(x) W_1^T + b_1) W_2^T + b_2 ([FD] Sec. 3.2).
+
+    With cfg.mlp_fp8 the two Linears multiply FP8 operands with static
+    per-tensor scales w[p + "fp8_sx"] (x) and w[p + "fp8_sh"] (hidden):
+      r  = 1 / sqrt(mean(x^2) + eps)                 per token
+      W1g = W_1 diag(g)       quantized with its own scale
+      h  = GELU(r (Q(x) W1g_q^T) + b_1)
+      y  = Q(h) W2_q^T + b_2
+    amax (calibration, unquantized MLP only): records the largest |x| and
+    |h| of the block under keys p + "x" and p + "h"."""
+    g = w[p + "norm2_g"]
+    if not getattr(cfg, "mlp_fp8", 0):
+        a = rms_norm(x, g, cfg.norm_eps)
+        h = gelu(linear(a, w[p + "w1"], w[p + "b1"]))
+        if amax is not None:
+            amax[p + "x"] = max(amax.get(p + "x", 0.0), float(np.max(np.abs(x))))
+            amax[p + "h"] = max(amax.get(p + "h", 0.0), float(np.max(np.abs(h))))
+        return linear(h, w[p + "w2"], w[p + "b2"])
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + cfg.norm_eps)
+    w1g = w[p + "w1"] * g[None, :]
+    w1q = quantize_weight(w1g, weight_scale(w1g))
+    w2q = quantize_weight(w[p + "w2"], weight_scale(w[p + "w2"]))
+    h = gelu(r * (quantize_act(x, float(w[p + "fp8_sx"])) @ w1q.T) + w[p + "b1"])
+    return quantize_act(h, float(w[p + "fp8_sh"])) @ w2q.T + w[p + "b2"]
 
 
 def rope_split(head_dim: int):
@@ -174,6 +259,7 @@ class OracleDecoder:
         n = np.arange(cfg.L_frm)
         self.row = (n // cfg.tok_w).astype(np.float64)   # token grid row i
         self.col = (n % cfg.tok_w).astype(np.float64)    # token grid column j
+        self.amax: Optional[Dict[str, float]] = None      # set by calibrate_fp8
         self.reset()
 
     # -- state -------------------------------------------------------------
@@ -229,10 +315,7 @@ class OracleDecoder:
             o[:, h] = attention(qh, np.concatenate(ks), np.concatenate(vs))
         x = x + linear(o.reshape(L, H * Dh), w[p + "wo"], w[p + "bo"])
         # pre-MLP RMSNorm, MLP with GELU, residual
-        a = rms_norm(x, w[p + "norm2_g"], cfg.norm_eps)
-        hdn = gelu(linear(a, w[p + "w1"], w[p + "b1"]))
-        x = x + linear(hdn, w[p + "w2"], w[p + "b2"])
-        return x
+        return x + mlp(cfg, w, p, x, self.amax)
 
     # -- one latent frame ----------------------------------------------------
     def embed(self, z_t: np.ndarray) -> np.ndarray:
@@ -288,6 +371,24 @@ class OracleDecoder:
         return self.cache[l][frames.index(frame)]
 
 
+def calibrate_fp8(cfg, weights, z: np.ndarray) -> Dict[str, float]:
+    """Static FP8 scales of every MLP layer ([FD] Sec. 4.6: static
+    calibration): stream the calibration frames z[0..T-1] through the decoder
+    with unquantized MLPs, take per block the largest |x| entering the MLP and
+    the largest |GELU output|, and set each scale to fp32(amax / 448), so the
+    calibration data never saturates. Returns {"b{l}.fp8_sx": s, "b{l}.fp8_sh":
+    s, ...}, with "r{l}.*" for the paper head's refinement blocks."""
+    dec = OracleDecoder(cfg.replace(mlp_fp8=0), weights)
+    dec.amax = {}
+    for t in range(z.shape[0]):
+        dec.decode_frame(z[t])
+    out = {}
+    for key, a in dec.amax.items():
+        p, kind = key[:-1], key[-1]
+        out[p + "fp8_s" + kind] = float(np.float32(a / E4M3_MAX)) if a > 0 else 1.0
+    return out
+
+
 def decode_video(cfg, weights, z: np.ndarray,
                  frames: Optional[int] = None) -> np.ndarray:
     """Stream frames z[0..T'-1] through a fresh decoder; stack the outputs
@@ -326,8 +427,7 @@ def _masked_block(cfg, w, p, x, tau, row, col, allowed):
         pr = pr / pr.sum(axis=-1, keepdims=True)
         o[:, h] = pr @ v[:, g]
     x = x + linear(o.reshape(S, H * Dh), w[p + "wo"], w[p + "bo"])
-    a = rms_norm(x, w[p + "norm2_g"], cfg.norm_eps)
-    return x + linear(gelu(linear(a, w[p + "w1"], w[p + "b1"])), w[p + "w2"], w[p + "b2"])
+    return x + mlp(cfg, w, p, x)
 
 
 def _window_mask(frame_of, span):

@@ -170,7 +170,38 @@ def test_rope_3d_parts_follow_their_own_axis():
 # The whole step against a composition of torch library routines
 # --------------------------------------------------------------------------
 
-def _torch_library_decoder(cfg, weights, z):
+def _torch_f8(t, s):
+    """Dequantized FP8 E4M3 value of t with scale s through torch's own
+    float8_e4m3fn cast (its rounding is an implementation independent of the
+    oracle's); the quotient is formed in float32, values must stay below 464
+    (torch turns larger ones into NaN instead of saturating)."""
+    q = (t.float() * torch.tensor(1.0 / float(s), dtype=torch.float64).float())
+    return q.to(torch.float8_e4m3fn).double() * float(s)
+
+
+def _torch_mlp(cfg, W, p, x, amax=None):
+    """MLP sublayer from torch calls; with cfg.mlp_fp8 the operands of both
+    Linears are FP8 (weights: per-tensor scale max|w|/448 in float32, the
+    RMSNorm gain folded into W_1 first; activations: the static scales)."""
+    g = W[p + "norm2_g"]
+    if not getattr(cfg, "mlp_fp8", 0):
+        a = F.rms_norm(x, (cfg.d_model,), g, eps=cfg.norm_eps)
+        h = F.gelu(F.linear(a, W[p + "w1"], W[p + "b1"]))
+        if amax is not None:
+            amax[p + "x"] = max(amax.get(p + "x", 0.0), float(x.abs().max()))
+            amax[p + "h"] = max(amax.get(p + "h", 0.0), float(h.abs().max()))
+        return F.linear(h, W[p + "w2"], W[p + "b2"])
+
+    def wq(w):
+        s = float(torch.tensor(float(w.abs().max()) / 448.0).float())
+        return (w / s).to(torch.float8_e4m3fn).double() * s
+
+    r = torch.rsqrt((x * x).mean(-1, keepdim=True) + cfg.norm_eps)
+    h = F.gelu(r * F.linear(_torch_f8(x, W[p + "fp8_sx"]), wq(W[p + "w1"] * g)) + W[p + "b1"])
+    return F.linear(_torch_f8(h, W[p + "fp8_sh"]), wq(W[p + "w2"]), W[p + "b2"])
+
+
+def _torch_library_decoder(cfg, weights, z, amax=None):
     """Full-sequence forward built from torch library calls (F.linear,
     F.rms_norm, F.scaled_dot_product_attention with a boolean mask, F.gelu,
     F.pixel_unshuffle / F.pixel_shuffle) and RoPE as complex multiplication
@@ -213,8 +244,7 @@ def _torch_library_decoder(cfg, weights, z):
         o = F.scaled_dot_product_attention(q.transpose(0, 1), k.transpose(0, 1),
                                            v.transpose(0, 1), attn_mask=mask)
         x = x + F.linear(o.transpose(0, 1).reshape(-1, H * Dh), W[p + "wo"], W[p + "bo"])
-        a = F.rms_norm(x, (cfg.d_model,), W[p + "norm2_g"], eps=cfg.norm_eps)
-        x = x + F.linear(F.gelu(F.linear(a, W[p + "w1"], W[p + "b1"])), W[p + "w2"], W[p + "b2"])
+        x = x + _torch_mlp(cfg, W, p, x, amax)
     y = F.linear(F.rms_norm(x, (cfg.d_model,), W["final_g"], eps=cfg.norm_eps),
                  W["out_w"], W["out_b"])
     y = y.view(T, cfg.tok_h, cfg.tok_w, cfg.c_out).permute(0, 3, 1, 2)
@@ -394,8 +424,7 @@ def _torch_library_paper_decoder(cfg, weights, z):
         o = F.scaled_dot_product_attention(q.transpose(0, 1), k.transpose(0, 1),
                                            v.transpose(0, 1), attn_mask=mask)
         x = x + F.linear(o.transpose(0, 1).reshape(-1, H * Dh), W[p + "wo"], W[p + "bo"])
-        a = F.rms_norm(x, (D,), W[p + "norm2_g"], eps=cfg.norm_eps)
-        return x + F.linear(F.gelu(F.linear(a, W[p + "w1"], W[p + "b1"])), W[p + "w2"], W[p + "b2"])
+        return x + _torch_mlp(cfg, W, p, x)
 
     zt = torch.from_numpy(np.asarray(z, np.float64))
     toks = F.pixel_unshuffle(zt, cfg.patch).flatten(2).transpose(1, 2).reshape(T * L, cfg.c_in)
