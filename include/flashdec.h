@@ -90,6 +90,17 @@ typedef struct {
                             sub-frames, then RMSNorm, Linear D -> D, GELU,
                             Linear D -> C P^2 and PixelShuffle per sub-frame    */
   int32_t n_refine;      /* refinement blocks (head_mode 1; 1 .. 8)              */
+  int32_t mlp_fp8;       /* 1: every Transformer block's MLP (backbone and
+                            refinement) multiplies FP8 E4M3 operands with static
+                            per-tensor scales (Sec. 4.6, optimization 4). Needs
+                            dtype BF16, d_model a multiple of 128 and
+                            fd_weights.mlp_scales. Weights are quantized here:
+                            W_1 diag(norm2_g) and W_2 each with the scale
+                            fp32(max|W| / 448), round to nearest even        */
+  int32_t record_mlp_amax; /* 1 (mlp_fp8 = 0 only): the MLP epilogues record,
+                            per block, max |x| entering the MLP and max |GELU
+                            output| since the last fd_reset; read them as
+                            static scales with fd_mlp_fp8_scales             */
 } fd_config;
 
 /*
@@ -114,6 +125,13 @@ typedef struct {
  *   sp1_w [D][D], sp1_b [D]             first spatial MLP layer
  *   out_w [C P^2][D], out_b [C P^2]     second layer, channel order (c, dy, dx)
  * (up_w .. sp1_b are ignored with head_mode 0.)
+ * With mlp_fp8 = 1:
+ *   mlp_scales[l] -> 2 floats {s_x, s_h}, one entry per block (backbone, then
+ *            refinement): static scales of the MLP input x and of the GELU
+ *            output h. x is stored as e4m3(x / s_x) before the RMSNorm row scale
+ *            (which, like the gain, multiplies the fp32 product), h as
+ *            e4m3(h / s_h); rounding to nearest even, saturating at +-448.
+ *            Ignored with mlp_fp8 = 0.
  */
 typedef struct {
   const float *embed_w, *embed_b;
@@ -123,6 +141,7 @@ typedef struct {
   const float *const *w1, *const *b1, *const *w2, *const *b2;
   const float *final_g, *out_w, *out_b;
   const float *up_w, *up_b, *sp1_w, *sp1_b;
+  const float *const *mlp_scales;
 } fd_weights;
 
 /*
@@ -203,6 +222,20 @@ FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
 
 /*
+ * Test/debug: run the second half of block `block` (backbone blocks first,
+ * then refinement blocks) once on a given residual stream: x_host [L_frm][D]
+ * fp32 becomes the stream, the attention output is set to zero, and the
+ * block's O-projection (so x + b_o), MLP-up and MLP-down kernels run with
+ * the handle's weights (FP8 with mlp_fp8); the resulting stream
+ * x + b_o + MLP(x + b_o) is copied to out_host [L_frm][D] fp32. Both sides of
+ * a parity test then quantize identical float32 inputs. Synchronous;
+ * overwrites the handle's per-frame scratch (not the ring cache), so it must
+ * not overlap a decode; records no calibration ranges.
+ */
+FD_API fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host,
+                                      float* out_host);
+
+/*
  * Kernel timing (requires cfg.kernel_timing = 1 or 2): waits for the last
  * enqueued frame and writes the device time in ms of each timed kernel of
  * that frame (every kernel, or every attention launch), in launch order, to
@@ -220,6 +253,19 @@ typedef enum {
 } fd_kernel_kind;
 FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out,
                                    int32_t cap, int32_t* n_out);
+
+/*
+ * Static FP8 scales from the calibration recorded by a handle created with
+ * record_mlp_amax = 1 ([FD] Sec. 4.6: static calibration): for every block
+ * (backbone, then refinement), scales_out[2 l] = fp32(max |x| / 448) and
+ * scales_out[2 l + 1] = fp32(max |h| / 448) over the frames decoded since the
+ * last fd_reset (1 where nothing was seen), ready for fd_weights.mlp_scales of
+ * an mlp_fp8 handle. *n_out = 2 * (n_blocks + n_refine); cap = 0 queries it.
+ * Synchronises the handle's last stream. FD_ERR_INVALID_ARG if the handle
+ * does not record.
+ */
+FD_API fd_status_t fd_mlp_fp8_scales(fd_handle* h, float* scales_out, int32_t cap,
+                                     int32_t* n_out);
 
 /*
  * Self-test of the device-side failure path (no handle needed; runs on the

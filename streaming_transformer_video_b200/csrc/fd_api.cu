@@ -95,13 +95,14 @@ fd_status_t get_encode() {
   return FD_OK;
 }
 
-// bf16 tensor map with 128-byte swizzle. dims/strides innermost first;
-// strides[i] is the byte pitch of dimension i+1.
+// Tensor map (bf16 by default, or bytes for E4M3) with 128-byte swizzle.
+// dims/strides innermost first; strides[i] is the byte pitch of dimension i+1.
 fd_status_t make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                      const uint64_t* strides, const uint32_t* box) {
+                      const uint64_t* strides, const uint32_t* box,
+                      CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   FD_TRY(get_encode());
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+  CUresult r = g_encode(m, type, rank, const_cast<void*>(base),
                         reinterpret_cast<const cuuint64_t*>(dims),
                         reinterpret_cast<const cuuint64_t*>(strides),
                         reinterpret_cast<const cuuint32_t*>(box), estr,
@@ -118,6 +119,35 @@ fd_status_t make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64
   const uint64_t strides[1] = {cols * 2};
   const uint32_t box[2] = {64, box_rows};
   return make_tmap(m, base, 2, dims, strides, box);
+}
+
+// Row-major [rows][cols] E4M3 matrix read in boxes of box_rows x 128 bytes.
+fd_status_t make_tmap_2d_e4m3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                              uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols};
+  const uint32_t box[2] = {128, box_rows};
+  return make_tmap(m, base, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8);
+}
+
+// FP8 E4M3 code of v: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits,
+// no infinities; the largest finite value 448 = 1.75 * 2^8 is code 0x7E and
+// 0x7F is NaN. Round to nearest, ties to even (the default rounding mode of
+// nearbyint); magnitudes >= 448 after rounding saturate to 448.
+uint8_t e4m3_encode(double v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(v);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int ex = 0;
+  std::frexp(a, &ex);                       // a = m 2^ex, m in [0.5, 1)
+  int e = std::max(ex - 1, -6);             // binade 2^e; subnormal spacing below 2^-6
+  double q = std::nearbyint(std::ldexp(a, 3 - e));   // multiples of 2^(e-3)
+  if (q >= 16.0) { q = 8.0; ++e; }          // rounded up into the next binade
+  if (e == -6 && q < 8.0) return sign | uint8_t(q);               // subnormal (or zero)
+  if (e > 8 || (e == 8 && q > 14.0)) return sign | 0x7E;          // beyond 448
+  return sign | uint8_t(((e + 7) << 3) | (int(q) - 8));
 }
 
 struct KernelLaunch {
@@ -162,6 +192,7 @@ struct fd_handle {
   fd_config cfg{};
   int bf = 0;                       // 1: bf16 storage + tcgen05 kernels
   int paper = 0;                    // 1: the paper's output head
+  int fp8 = 0;                      // 1: FP8 E4M3 MLP GEMMs
   int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
   int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
@@ -180,6 +211,12 @@ struct fd_handle {
   float *bup = nullptr, *bsp1 = nullptr;
   void *kc = nullptr, *vtc = nullptr;
   void *rkc = nullptr, *rvtc = nullptr;     // refinement ring (paper head)
+  // FP8 MLP: per block (backbone, then refinement) static activation scales
+  // and per-tensor weight scales; x8 = E4M3 copy of x for the MLP-up
+  std::vector<float> s_x, s_h, s_w1, s_w2;
+  void* x8 = nullptr;
+  unsigned* amax = nullptr;                 // calibration: [blocks][2] float bits
+  int n_amax = 0;
   float *x32 = nullptr, *ssq = nullptr;
   float *xs32 = nullptr, *xss = nullptr;    // [r_t][L][D], [r_t][L][D/32]
   void* xsb = nullptr;                      // [r_t][L][D] storage type
@@ -192,7 +229,7 @@ struct fd_handle {
 
   // TMA maps (bf16 path)
   CUtensorMap tm_xb{}, tm_o{}, tm_h{}, tm_q{}, tm_k{}, tm_v{}, tm_wout{};
-  CUtensorMap tm_rk{}, tm_rv{}, tm_wup{}, tm_wsp1{}, tm_hs{};
+  CUtensorMap tm_rk{}, tm_rv{}, tm_wup{}, tm_wsp1{}, tm_hs{}, tm_x8{}, tm_h8{};
   std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_w1, tm_w2, tm_xs;
 
   // graph
@@ -235,6 +272,23 @@ struct fd_handle {
     FD_TRY(upload(&d, src, n * 4));
     *dst = static_cast<float*>(d);
     return FD_OK;
+  }
+  // Weight [rows][cols] with optional per-column gain folded in, quantized to
+  // E4M3 with the per-tensor scale fp32(max|w g| / 448) (returned in *scale).
+  fd_status_t upload_w_e4m3(void** dst, const float* w, size_t rows, size_t cols,
+                            const float* gain, float* scale) {
+    std::vector<double> v(rows * cols);
+    double amax = 0.0;
+    for (size_t r = 0; r < rows; ++r)
+      for (size_t c = 0; c < cols; ++c) {
+        v[r * cols + c] = double(w[r * cols + c]) * (gain ? double(gain[c]) : 1.0);
+        amax = std::max(amax, std::fabs(v[r * cols + c]));
+      }
+    const float s = amax > 0.0 ? float(amax / 448.0) : 1.f;
+    std::vector<uint8_t> q(rows * cols);
+    for (size_t i = 0; i < q.size(); ++i) q[i] = e4m3_encode(v[i] / double(s));
+    *scale = s;
+    return upload(dst, q.data(), q.size());
   }
   // Weight [rows][cols] with optional per-column gain folded in, in storage type.
   fd_status_t upload_w(void** dst, const float* w, size_t rows, size_t cols, const float* gain) {
@@ -303,9 +357,10 @@ struct fd_handle {
   fd_status_t build_graph();
   fd_status_t add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, const void* A,
                        const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
-                       cudaGraphNode_t* node);
+                       cudaGraphNode_t* node, bool f8 = false);
   fd_status_t add_out_gemm(OutNode on, int N);
   fd_status_t add_block(int wi, const BlockIO& io);
+  fd_status_t add_post_attention(int wi, const BlockIO& io);
   EpiParams base_epi(const BlockIO& io) const;
   BlockIO backbone_io(int layer);
   BlockIO subframe_io(int tau, int layer);
@@ -315,11 +370,11 @@ namespace {
 
 bool valid_handle(const fd_handle* h) { return h && h->magic == kMagic; }
 
-template <int BN, int KIND>
+template <int BN, int KIND, bool F8>
 fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   using S = TcGemmSmem<BN, STAGES>;
-  const void* f = reinterpret_cast<const void*>(&tc_gemm_kernel<BN, STAGES, KIND, 64>);
+  const void* f = reinterpret_cast<const void*>(&tc_gemm_kernel<BN, STAGES, KIND, 64, F8>);
   FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc));
   const int tiles = ((M + 127) / 128) * (N / BN);
   k->func = f;
@@ -329,12 +384,12 @@ fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   return FD_OK;
 }
 
-template <int KIND>
+template <int KIND, bool F8 = false>
 fd_status_t tc_gemm_pick(int M, int N, int num_sms, int* bn, KernelLaunch* k) {
-  if (N % 256 == 0) { *bn = 256; return tc_gemm_launch<256, KIND>(M, N, num_sms, k); }
-  if (N % 128 == 0) { *bn = 128; return tc_gemm_launch<128, KIND>(M, N, num_sms, k); }
+  if (N % 256 == 0) { *bn = 256; return tc_gemm_launch<256, KIND, F8>(M, N, num_sms, k); }
+  if (N % 128 == 0) { *bn = 128; return tc_gemm_launch<128, KIND, F8>(M, N, num_sms, k); }
   *bn = 64;
-  return tc_gemm_launch<64, KIND>(M, N, num_sms, k);
+  return tc_gemm_launch<64, KIND, F8>(M, N, num_sms, k);
 }
 
 template <int KIND>
@@ -372,6 +427,8 @@ EpiParams fd_handle::base_epi(const BlockIO& io) const {
   e.out_bf16 = cfg.io_dtype == FD_BF16;
   e.pl_mul = 1;
   e.pl_add = 0;
+  e.acc_scale = 1.f;
+  e.q_inv = 1.f;
   return e;
 }
 
@@ -391,16 +448,20 @@ BlockIO fd_handle::subframe_io(int tau, int layer) {
 // copies the pointed-to values, so stack storage inside one call suffices.
 fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, const void* A,
                                 const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
-                                cudaGraphNode_t* node) {
+                                cudaGraphNode_t* node, bool f8) {
   ep.N = N;
   KernelLaunch k{};
   if (bf) {
     int bn = 0;
-    switch (kind) {
+    if (f8) {                     // FP8 MLP: the two MLP GEMMs
+      if (kind == EPI_GELU_Q) FD_TRY((tc_gemm_pick<EPI_GELU_Q, true>(L, N, num_sms, &bn, &k)));
+      else FD_TRY((tc_gemm_pick<EPI_RESID, true>(L, N, num_sms, &bn, &k)));
+    } else switch (kind) {
       case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(L, N, num_sms, &bn, &k)); break;
       case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(L, N, num_sms, &bn, &k)); break;
       case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(L, N, num_sms, &bn, &k)); break;
       case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(L, N, num_sms, &bn, &k)); break;
+      case EPI_RESID_Q: FD_TRY(tc_gemm_pick<EPI_RESID_Q>(L, N, num_sms, &bn, &k)); break;
       default: FD_TRY(tc_gemm_pick<EPI_FINAL>(L, N, num_sms, &bn, &k)); break;
     }
     CUtensorMap a = tmA, b = tmB;
@@ -497,15 +558,47 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     void* args[] = {&ap};
     FD_TRY(add_kernel(k, args));
   }
+  return add_post_attention(wi, io);
+}
+
+// The rest of a block after its attention: O-projection (+residual), MLP-up
+// (+RMSNorm, GELU), MLP-down (+residual); FP8 E4M3 MLP with mlp_fp8.
+fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
+  const int D = cfg.d_model, H = cfg.n_heads, Dh = cfg.head_dim;
+  EpiParams e;
+  if (fp8) {
+    // output projection + residual; x also stored as e4m3(x / s_x)
+    e = base_epi(io);
+    e.bias = bo[wi];
+    e.x8 = x8;
+    e.q_inv = float(1.0 / double(s_x[wi]));
+    FD_TRY(add_gemm(EPI_RESID_Q, FD_K_OPROJ, tm_o, o, tm_wo[wi], wo[wi], D, H * Dh, e, nullptr));
+    // FP8 MLP up: h = GELU(r (x8 W1q^T) s_x s_w1 + b_1) stored as e4m3(h / s_h)
+    e = base_epi(io);
+    e.bias = b1[wi];
+    e.hout = hb;
+    e.acc_scale = float(double(s_x[wi]) * double(s_w1[wi]));
+    e.q_inv = float(1.0 / double(s_h[wi]));
+    FD_TRY(add_gemm(EPI_GELU_Q, FD_K_MLP_UP, tm_x8, x8, tm_w1[wi], w1[wi], dff, D, e, nullptr,
+                    true));
+    // FP8 MLP down + residual: x += (h8 W2q^T) s_h s_w2 + b_2
+    e = base_epi(io);
+    e.bias = b2[wi];
+    e.acc_scale = float(double(s_h[wi]) * double(s_w2[wi]));
+    return add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h8, hb, tm_w2[wi], w2[wi], D, dff, e, nullptr,
+                    true);
+  }
   // output projection + residual
   e = base_epi(io);
   e.bias = bo[wi];
+  if (amax) e.amax = amax + 2 * wi;               // calibration: max |x| entering the MLP
   FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[wi] : tm_o, wo[wi], D, H * Dh, e,
                   nullptr));
   // MLP up + GELU
   e = base_epi(io);
   e.bias = b1[wi];
   e.hout = hb;
+  if (amax) e.amax = amax + 2 * wi + 1;           // calibration: max |GELU output|
   FD_TRY(add_gemm(EPI_GELU, FD_K_MLP_UP, *io.tm_x, io.xb, bf ? tm_w1[wi] : *io.tm_x, w1[wi], dff,
                   D, e, nullptr));
   // MLP down + residual
@@ -661,6 +754,12 @@ fd_status_t validate(const fd_config* c) {
     return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0, 1 or 2");
   if (c->head_mode != 0 && c->head_mode != 1)
     return fail(FD_ERR_INVALID_ARG, "config: head_mode must be 0 or 1");
+  if ((c->mlp_fp8 != 0 && c->mlp_fp8 != 1) || (c->record_mlp_amax != 0 && c->record_mlp_amax != 1))
+    return fail(FD_ERR_INVALID_ARG, "config: mlp_fp8 and record_mlp_amax must be 0 or 1");
+  if (c->mlp_fp8 && (c->dtype != FD_BF16 || c->d_model % 128))
+    return fail(FD_ERR_UNSUPPORTED, "config: mlp_fp8 needs dtype bf16 and d_model a multiple of 128");
+  if (c->mlp_fp8 && c->record_mlp_amax)
+    return fail(FD_ERR_INVALID_ARG, "config: record_mlp_amax calibrates the unquantized MLP (mlp_fp8 0)");
   if (c->head_mode == 1) {
     if (c->n_refine < 1 || c->n_refine > 8)
       return fail(FD_ERR_UNSUPPORTED, "config: n_refine must be 1 .. 8 (got %d)", c->n_refine);
@@ -678,6 +777,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   const fd_config& c = *cfg;
   h->bf = c.dtype == FD_BF16;
   h->paper = c.head_mode == 1;
+  h->fp8 = c.mlp_fp8;
   h->elt = h->bf ? 2 : 4;
   h->io_elt = c.io_dtype == FD_BF16 ? 2 : 4;
   h->tok_h = c.grid_h / c.patch;
@@ -720,8 +820,18 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     void* p;
     FD_TRY(h->upload_w(&p, w->wqkv[l], h->qkv, D, w->norm1_g[l])); h->wqkv.push_back(p);
     FD_TRY(h->upload_w(&p, w->wo[l], D, size_t(H) * Dh, nullptr)); h->wo.push_back(p);
-    FD_TRY(h->upload_w(&p, w->w1[l], h->dff, D, w->norm2_g[l])); h->w1.push_back(p);
-    FD_TRY(h->upload_w(&p, w->w2[l], D, h->dff, nullptr)); h->w2.push_back(p);
+    if (h->fp8) {
+      float s1 = 1.f, s2 = 1.f;
+      FD_TRY(h->upload_w_e4m3(&p, w->w1[l], h->dff, D, w->norm2_g[l], &s1)); h->w1.push_back(p);
+      FD_TRY(h->upload_w_e4m3(&p, w->w2[l], D, h->dff, nullptr, &s2)); h->w2.push_back(p);
+      h->s_w1.push_back(s1);
+      h->s_w2.push_back(s2);
+      h->s_x.push_back(w->mlp_scales[l][0]);
+      h->s_h.push_back(w->mlp_scales[l][1]);
+    } else {
+      FD_TRY(h->upload_w(&p, w->w1[l], h->dff, D, w->norm2_g[l])); h->w1.push_back(p);
+      FD_TRY(h->upload_w(&p, w->w2[l], D, h->dff, nullptr)); h->w2.push_back(p);
+    }
     float* f;
     FD_TRY(h->upload_f32(&f, w->bqkv[l], h->qkv)); h->bqkv.push_back(f);
     FD_TRY(h->upload_f32(&f, w->bo[l], D)); h->bo.push_back(f);
@@ -770,6 +880,11 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(h->alloc(&h->xsb, size_t(c.r_t) * L * D * h->elt));
     FD_TRY(h->alloc(&h->xss, size_t(c.r_t) * L * (D / 32) * 4));
   }
+  if (h->fp8) FD_TRY(h->alloc(&h->x8, L * D));
+  if (c.record_mlp_amax) {
+    h->n_amax = 2 * (NB + NR);
+    FD_TRY(h->alloc(&h->amax, size_t(h->n_amax) * 4));
+  }
   FD_TRY(h->alloc(&h->ctr, 64));
   FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * (1 + (h->paper ? c.r_t : 0))));
   FD_TRY(h->alloc(&h->status, 16));
@@ -806,8 +921,17 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
       CUtensorMap m;
       FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(h->qkv))); h->tm_wqkv.push_back(m);
       FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D))); h->tm_wo.push_back(m);
-      FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
-      FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+      if (h->fp8) {
+        FD_TRY(make_tmap_2d_e4m3(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
+        FD_TRY(make_tmap_2d_e4m3(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+      } else {
+        FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
+        FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+      }
+    }
+    if (h->fp8) {
+      FD_TRY(make_tmap_2d_e4m3(&h->tm_x8, h->x8, L, D, 128));
+      FD_TRY(make_tmap_2d_e4m3(&h->tm_h8, h->hb, L, h->dff, 128));   // hidden as E4M3 [L][4D]
     }
     const int n_out = h->paper ? c_px : h->c_out;
     FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, n_out, D, bn_of(n_out)));
@@ -858,6 +982,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   }
   FD_CUDA(cudaMemset(h->ctr, 0, 64));
   FD_CUDA(cudaMemset(h->status, 0, 16));
+  if (h->amax) FD_CUDA(cudaMemset(h->amax, 0, size_t(h->n_amax) * 4));
   FD_CUDA(cudaMemset(h->fs, 0, sizeof(FrameState)));
   FD_TRY(h->build_graph());
   FD_CUDA(cudaDeviceSynchronize());
@@ -926,6 +1051,14 @@ fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle
         !w->norm2_g[l] || !w->w1[l] || !w->b1[l] || !w->w2[l] || !w->b2[l] ||
         (cfg->kv_norm && (!w->knorm_g[l] || !w->vnorm_g[l])))
       return fail(FD_ERR_INVALID_ARG, "fd_create: null weight pointer in block %d", l);
+  if (cfg->mlp_fp8) {
+    if (!w->mlp_scales) return fail(FD_ERR_INVALID_ARG, "fd_create: mlp_fp8 needs mlp_scales");
+    for (int l = 0; l < n_all; ++l) {
+      const float* sc = w->mlp_scales[l];
+      if (!sc || !(sc[0] > 0.f) || !(sc[1] > 0.f) || !std::isfinite(sc[0]) || !std::isfinite(sc[1]))
+        return fail(FD_ERR_INVALID_ARG, "fd_create: FP8 scales of block %d must be finite and > 0", l);
+    }
+  }
   fd_handle* h = new (std::nothrow) fd_handle();
   if (!h) return fail(FD_ERR_OOM, "fd_create: host allocation failed");
   const fd_status_t s = create_impl(cfg, weights, h);
@@ -950,6 +1083,7 @@ fd_status_t fd_reset(fd_handle* h, void* stream) {
   }
   FD_CUDA(cudaMemsetAsync(h->ctr, 0, 64, s));
   FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
+  if (h->amax) FD_CUDA(cudaMemsetAsync(h->amax, 0, size_t(h->n_amax) * 4, s));
   h->last_stream = s;
   return FD_OK;
 }
@@ -1077,6 +1211,71 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
               h->bf ? bf16_bits_to_f32(reinterpret_cast<uint16_t*>(rows.data())[n2])
                     : reinterpret_cast<float*>(rows.data())[n2];
       }
+  }
+  return FD_OK;
+}
+
+fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, float* out_host) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_block_mlp: invalid handle");
+  const fd_config& c = h->cfg;
+  const int n_all = c.n_blocks + (h->paper ? c.n_refine : 0);
+  if (block < 0 || block >= n_all || !x_host || !out_host)
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_block_mlp: bad block or null buffer");
+  FD_CUDA(cudaDeviceSynchronize());
+  const size_t n = size_t(h->L) * c.d_model;
+  FD_CUDA(cudaMemcpy(h->x32, x_host, n * 4, cudaMemcpyHostToDevice));
+  FD_CUDA(cudaMemset(h->o, 0, size_t(h->L) * c.n_heads * c.head_dim * h->elt));
+  // a one-off graph of the block's post-attention kernels on the backbone
+  // stream; no timing events, no calibration records
+  cudaGraph_t saved_graph = h->graph;
+  cudaGraphNode_t saved_last = h->last_node;
+  const size_t saved_kinds = h->kinds.size();
+  const int saved_timing = h->cfg.kernel_timing;
+  unsigned* saved_amax = h->amax;
+  cudaGraph_t g = nullptr;
+  cudaGraphExec_t ex = nullptr;
+  FD_CUDA(cudaGraphCreate(&g, 0));
+  h->graph = g;
+  h->last_node = nullptr;
+  h->cfg.kernel_timing = 0;
+  h->amax = nullptr;
+  fd_status_t st = h->add_post_attention(block, h->backbone_io(0));
+  h->graph = saved_graph;
+  h->last_node = saved_last;
+  h->kinds.resize(saved_kinds);
+  h->cfg.kernel_timing = saved_timing;
+  h->amax = saved_amax;
+  cudaError_t e = cudaSuccess;
+  if (st == FD_OK) e = cudaGraphInstantiate(&ex, g, 0);
+  if (st == FD_OK && e == cudaSuccess) e = cudaGraphLaunch(ex, nullptr);
+  if (st == FD_OK && e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
+  if (st == FD_OK && e == cudaSuccess)
+    e = cudaMemcpy(out_host, h->x32, n * 4, cudaMemcpyDeviceToHost);
+  if (ex) cudaGraphExecDestroy(ex);
+  cudaGraphDestroy(g);
+  if (st == FD_OK && e != cudaSuccess) {
+    cudaGetLastError();
+    st = fail(FD_ERR_CUDA, "fd_debug_block_mlp: %s", cudaGetErrorString(e));
+  }
+  return st;
+}
+
+fd_status_t fd_mlp_fp8_scales(fd_handle* h, float* scales_out, int32_t cap, int32_t* n_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_mlp_fp8_scales: invalid handle");
+  if (!n_out) return fail(FD_ERR_INVALID_ARG, "fd_mlp_fp8_scales: null n_out");
+  if (!h->amax)
+    return fail(FD_ERR_INVALID_ARG, "fd_mlp_fp8_scales: handle created without record_mlp_amax");
+  *n_out = h->n_amax;
+  if (cap == 0) return FD_OK;
+  if (!scales_out || cap < h->n_amax)
+    return fail(FD_ERR_INVALID_ARG, "fd_mlp_fp8_scales: output array too small");
+  FD_CUDA(cudaStreamSynchronize(h->last_stream));
+  std::vector<unsigned> bits(h->n_amax);
+  FD_CUDA(cudaMemcpy(bits.data(), h->amax, bits.size() * 4, cudaMemcpyDeviceToHost));
+  for (int i = 0; i < h->n_amax; ++i) {
+    float a;
+    std::memcpy(&a, &bits[i], 4);
+    scales_out[i] = a > 0.f ? float(double(a) / 448.0) : 1.f;
   }
   return FD_OK;
 }

@@ -13,6 +13,14 @@
 //   UP     bias -> temporal upsampling (Sec. 3.4, Eq. 3): output channels
 //          [tau D, (tau+1) D) become the residual stream of sub-frame tau
 //          (fp32 copy, storage-type copy, per-32-column sums of squares)
+// FP8 MLP (Sec. 4.6, static per-tensor scales):
+//   RESID_Q  as RESID, but the copy of x is FP8 E4M3, x / s_x (the MLP-up's
+//            A operand), instead of the storage type
+//   GELU_Q   dequantize (acc s_x s_w1) + RMSNorm row scale + bias + GELU ->
+//            FP8 hidden h / s_h (the MLP-down's A operand)
+//   RESID with acc_scale = s_h s_w2 dequantizes the MLP-down product
+// Calibration (unquantized path): RESID and GELU can record max |value| of
+// their outputs into a device word (float bits, atomicMax).
 //
 // RMSNorm fusion: the gain g is folded into the following weight matrix at
 // create time, so RMSNorm(x) W^T = diag(r) (x (W diag g)^T) with
@@ -24,12 +32,15 @@
 
 namespace fd {
 
-enum EpiKind { EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2, EPI_FINAL = 3, EPI_UP = 4 };
+enum EpiKind {
+  EPI_QKV = 0, EPI_RESID = 1, EPI_GELU = 2, EPI_FINAL = 3, EPI_UP = 4,
+  EPI_RESID_Q = 5, EPI_GELU_Q = 6
+};
 
 // Kinds whose A operand is an RMSNorm input (their rows get the row scale);
 // a null EpiParams::ssq turns the scale off (the spatial MLP's second layer).
 constexpr bool epi_normed(int kind) {
-  return kind == EPI_QKV || kind == EPI_GELU || kind == EPI_FINAL;
+  return kind == EPI_QKV || kind == EPI_GELU || kind == EPI_FINAL || kind == EPI_GELU_Q;
 }
 
 struct EpiParams {
@@ -69,7 +80,38 @@ struct EpiParams {
   int tok_h;
   int pl_mul, pl_add;    // column block c = col / P^2 goes to pixel frame
                          // c * pl_mul + pl_add of the [C * r_t] output frames
+  // FP8 MLP
+  float acc_scale;       // dequantization of the accumulator (1: none)
+  float q_inv;           // 1 / static scale of the FP8 output
+  void* x8;              // RESID_Q: [M][D] E4M3 copy of x
+  // calibration: max |output| as float bits (null: off)
+  unsigned* amax;
 };
+
+// 64 floats * q_inv -> 64 E4M3 bytes (round to nearest even, saturating at
+// +-448), as four 16-byte stores.
+__device__ __forceinline__ void store_e4m3_64(uint8_t* dst, const float* v, float q_inv) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[c + 4 * i] * q_inv, v[c + 4 * i + 1] * q_inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[c + 4 * i + 2] * q_inv, v[c + 4 * i + 3] * q_inv), __NV_SATFINITE, __NV_E4M3);
+      w[i] = uint32_t(lo) | (uint32_t(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+__device__ __forceinline__ void record_amax(unsigned* amax, const float* v) {
+  float m = 0.f;
+#pragma unroll
+  for (int c = 0; c < 64; ++c) m = fmaxf(m, fabsf(v[c]));
+  atomicMax(amax, __float_as_uint(m));     // non-negative floats order as their bits
+}
 
 __device__ __forceinline__ float row_scale(const EpiParams& p, int row) {
   // ssq_parts = D / 32 is even (D is a multiple of 64): independent loads in
@@ -167,19 +209,24 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
         for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch] = from_f<T>(v[d]);
       }
     }
-  } else if constexpr (KIND == EPI_RESID) {
+  } else if constexpr (KIND == EPI_RESID || KIND == EPI_RESID_Q) {
     float* x = p.x32 + size_t(row) * p.D + col0;
+    const float sc = p.acc_scale;
 #pragma unroll
     for (int c = 0; c < 64; c += 4) {
       float4 o = *reinterpret_cast<const float4*>(x + c);
-      o.x += acc[c + 0] + __ldg(p.bias + col0 + c + 0);
-      o.y += acc[c + 1] + __ldg(p.bias + col0 + c + 1);
-      o.z += acc[c + 2] + __ldg(p.bias + col0 + c + 2);
-      o.w += acc[c + 3] + __ldg(p.bias + col0 + c + 3);
+      o.x += acc[c + 0] * sc + __ldg(p.bias + col0 + c + 0);
+      o.y += acc[c + 1] * sc + __ldg(p.bias + col0 + c + 1);
+      o.z += acc[c + 2] * sc + __ldg(p.bias + col0 + c + 2);
+      o.w += acc[c + 3] * sc + __ldg(p.bias + col0 + c + 3);
       *reinterpret_cast<float4*>(x + c) = o;
       acc[c + 0] = o.x; acc[c + 1] = o.y; acc[c + 2] = o.z; acc[c + 3] = o.w;
     }
-    store_vec<T, 64>(static_cast<T*>(p.xb) + size_t(row) * p.D + col0, acc);
+    if constexpr (KIND == EPI_RESID_Q)
+      store_e4m3_64(static_cast<uint8_t*>(p.x8) + size_t(row) * p.D + col0, acc, p.q_inv);
+    else
+      store_vec<T, 64>(static_cast<T*>(p.xb) + size_t(row) * p.D + col0, acc);
+    if (p.amax) record_amax(p.amax, acc);
     const int parts = p.D / 32;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -192,6 +239,12 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
 #pragma unroll
     for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * rs + __ldg(p.bias + col0 + c));
     store_vec<T, 64>(static_cast<T*>(p.hout) + size_t(row) * p.N + col0, acc);
+    if (p.amax) record_amax(p.amax, acc);
+  } else if constexpr (KIND == EPI_GELU_Q) {
+    const float sc = rs * p.acc_scale;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * sc + __ldg(p.bias + col0 + c));
+    store_e4m3_64(static_cast<uint8_t*>(p.hout) + size_t(row) * p.N + col0, acc, p.q_inv);
   } else if constexpr (KIND == EPI_UP) {
     const int tau = col0 / p.D, c0 = col0 - tau * p.D;
     const size_t r = size_t(tau) * p.M + row;             // row of sub-frame tau

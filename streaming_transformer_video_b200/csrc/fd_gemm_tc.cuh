@@ -1,13 +1,15 @@
 // fd_gemm_tc.cuh — persistent tcgen05 GEMM with fused epilogues (sm_100a).
 //
 //   C[M][N] = A[M][K] * B[N][K]^T     A, B bf16 (K contiguous), fp32 accumulate
+//                                     (F8: A, B FP8 E4M3, kind::f8f6f4)
 //
 // Used for every dense contraction of the FlashDecoder block (QKV, output
 // projection, both MLP layers) and the final projection. Structure:
-//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 per stage,
-//               128-byte swizzle, one mbarrier (expect_tx) per stage
+//   warp 0      TMA producer: A tile 128 x 128 bytes and B tile BN x 128 bytes
+//               per stage (64 bf16 or 128 E4M3 of K), 128-byte swizzle, one
+//               mbarrier (expect_tx) per stage
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=BN,
-//               K=16 per instruction, 4 per 64-wide stage) and commits
+//               32 bytes of K per instruction, 4 per stage) and commits
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, one
 //               token row per thread, fused epilogue (fd_epilogue.cuh)
 //               (eight epilogue warps, two per row group, measured no faster)
@@ -36,7 +38,7 @@ struct TcGemmSmem {
 constexpr int kEpiThreads = 128;                       // 4 epilogue warps
 constexpr int kGemmThreads = 64 + kEpiThreads;
 
-template <int BN, int STAGES, int KIND, int DH>
+template <int BN, int STAGES, int KIND, int DH, bool F8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int K, EpiParams ep, int* status) {
@@ -44,7 +46,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   constexpr uint32_t kTmemCols = 2 * BN;              // power of two: 128, 256 or 512
   static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM columns must be a power of 2");
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, BN);
+  constexpr uint32_t kIdesc = F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN);
+  constexpr int kBK = F8 ? 128 : 64;                  // K elements per stage (128 bytes)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -59,7 +62,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = ep.M;
   const int n_m = (M + 127) / 128, n_n = ep.N / BN;
-  const int n_tiles = n_m * n_n, k_blocks = K / 64;
+  const int n_tiles = n_m * n_n, k_blocks = K / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -84,8 +87,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, status)) goto producer_done;
           uint8_t* sa = smem + stage * S::kStage;
           mbar_arrive_expect_tx(&full[stage], S::kStage);
-          tma_load_2d(sa, &tmA, kb * 64, m_blk * 128, &full[stage]);
-          tma_load_2d(sa + S::kATile, &tmB, kb * 64, n_blk * BN, &full[stage]);
+          tma_load_2d(sa, &tmA, kb * kBK, m_blk * 128, &full[stage]);
+          tma_load_2d(sa + S::kATile, &tmB, kb * kBK, n_blk * BN, &full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -108,8 +111,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t adesc = sw128_desc(sa);
           const uint64_t bdesc = sw128_desc(sa + S::kATile);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)       // 16 bf16 = 32 bytes = 2 descriptor units
-            tc_mma_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {     // 32 bytes of K = 2 descriptor units
+            if constexpr (F8)
+              tc_mma_ss_f8(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0);
+            else
+              tc_mma_ss(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0);
+          }
           tc_commit(&empty[stage]);         // stage reusable once these MMAs finish
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }

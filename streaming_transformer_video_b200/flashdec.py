@@ -27,7 +27,7 @@ HEAD_MODES = {"linear": 0, "paper": 1}
 EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
            "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
-           "fd_selftest_wait_timeout"]
+           "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -37,7 +37,8 @@ class FDConfigC(ctypes.Structure):
         "kv_norm", "dtype", "io_dtype")] + [
         ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
         ("kernel_timing", ctypes.c_int32), ("head_mode", ctypes.c_int32),
-        ("n_refine", ctypes.c_int32)]
+        ("n_refine", ctypes.c_int32), ("mlp_fp8", ctypes.c_int32),
+        ("record_mlp_amax", ctypes.c_int32)]
 
 
 _PF = ctypes.POINTER(ctypes.c_float)
@@ -51,7 +52,8 @@ class FDWeightsC(ctypes.Structure):
                 ("wo", _PPF), ("bo", _PPF), ("norm2_g", _PPF),
                 ("w1", _PPF), ("b1", _PPF), ("w2", _PPF), ("b2", _PPF),
                 ("final_g", _PF), ("out_w", _PF), ("out_b", _PF),
-                ("up_w", _PF), ("up_b", _PF), ("sp1_w", _PF), ("sp1_b", _PF)]
+                ("up_w", _PF), ("up_b", _PF), ("sp1_w", _PF), ("sp1_b", _PF),
+                ("mlp_scales", _PPF)]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -79,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_last_step_kernel_ms.argtypes = [vp, _PF, ctypes.POINTER(i32), i32,
                                            ctypes.POINTER(i32)]
     lib.fd_selftest_wait_timeout.argtypes = [i32]
+    lib.fd_mlp_fp8_scales.argtypes = [vp, _PF, i32, ctypes.POINTER(i32)]
+    lib.fd_debug_block_mlp.argtypes = [vp, i32, _PF, _PF]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
             getattr(lib, name).restype = i32
@@ -122,7 +126,8 @@ def selftest_wait_timeout(timeout_us: int) -> int:
     return int(lib().fd_selftest_wait_timeout(int(timeout_us)))
 
 
-def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
+def make_config(cfg, io_dtype=None, kernel_timing: bool = False,
+                record_mlp_amax: bool = False) -> FDConfigC:
     """fd_config from any object with the decoder's shape attributes."""
     c = FDConfigC()
     for n in ("latent_ch", "grid_h", "grid_w", "patch", "d_model", "n_heads", "n_kv_heads",
@@ -137,6 +142,8 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False) -> FDConfigC:
     c.kernel_timing = int(kernel_timing)
     c.head_mode = HEAD_MODES[getattr(cfg, "head", "linear")]
     c.n_refine = int(getattr(cfg, "n_refine", 0)) if c.head_mode else 0
+    c.mlp_fp8 = int(getattr(cfg, "mlp_fp8", 0))
+    c.record_mlp_amax = int(record_mlp_amax)
     return c
 
 
@@ -158,13 +165,19 @@ class FlashDecoder:
     "b{l}.w1", "b{l}.b1", "b{l}.w2", "b{l}.b2", "final_g", "out_w", "out_b".
     With cfg.head == "paper" also "up_w", "up_b", "sp1_w", "sp1_b" and the
     refinement blocks "r{l}.*" (same keys as "b{l}.*"), l < cfg.n_refine.
+    With cfg.mlp_fp8 also the static FP8 scales "b{l}.fp8_sx", "b{l}.fp8_sh"
+    (and "r{l}.*") of every block, e.g. from mlp_fp8_scales() of a handle
+    created with record_mlp_amax=True.
     """
 
     def __init__(self, cfg, weights: Dict[str, np.ndarray], io_dtype=None,
-                 kernel_timing: bool = False):
+                 kernel_timing: bool = False, record_mlp_amax: bool = False):
         self._lib = lib()
         self.cfg = cfg
-        self.c = make_config(cfg, io_dtype, kernel_timing)
+        self.c = make_config(cfg, io_dtype, kernel_timing, record_mlp_amax)
+        self._prefixes = [f"b{l}." for l in range(cfg.n_blocks)]
+        if self.c.head_mode:
+            self._prefixes += [f"r{l}." for l in range(cfg.n_refine)]
         keep: List[np.ndarray] = []
 
         def fp(name):
@@ -172,9 +185,7 @@ class FlashDecoder:
             keep.append(a)
             return a.ctypes.data_as(_PF)
 
-        prefixes = [f"b{l}." for l in range(cfg.n_blocks)]
-        if self.c.head_mode:
-            prefixes += [f"r{l}." for l in range(cfg.n_refine)]
+        prefixes = self._prefixes
 
         def per_block(key):
             arr = (_PF * len(prefixes))(*[fp(p + key) for p in prefixes])
@@ -190,6 +201,15 @@ class FlashDecoder:
         if self.c.head_mode:
             w.up_w, w.up_b, w.sp1_w, w.sp1_b = (fp("up_w"), fp("up_b"), fp("sp1_w"),
                                                 fp("sp1_b"))
+        if self.c.mlp_fp8:
+            pairs = []
+            for p in prefixes:
+                a = np.array([weights[p + "fp8_sx"], weights[p + "fp8_sh"]], dtype=np.float32)
+                keep.append(a)
+                pairs.append(a.ctypes.data_as(_PF))
+            arr = (_PF * len(pairs))(*pairs)
+            keep.append(arr)
+            w.mlp_scales = ctypes.cast(arr, _PPF)
         h = ctypes.c_void_p()
         _check(self._lib.fd_create(ctypes.byref(self.c), ctypes.byref(w), ctypes.byref(h)),
                "fd_create")
@@ -258,6 +278,28 @@ class FlashDecoder:
         _check(self._lib.fd_debug_read_slot(self.h, block, slot, kv, out.ctypes.data_as(_PF)),
                "fd_debug_read_slot")
         return out
+
+    def debug_block_mlp(self, block: int, x: np.ndarray) -> np.ndarray:
+        """x + b_o + MLP(x + b_o) of block `block` for a residual stream x
+        [L_frm][D] (float32), through the block's own kernels."""
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        out = np.empty_like(x)
+        _check(self._lib.fd_debug_block_mlp(self.h, block, x.ctypes.data_as(_PF),
+                                            out.ctypes.data_as(_PF)), "fd_debug_block_mlp")
+        return out
+
+    def mlp_fp8_scales(self) -> Dict[str, float]:
+        """Static FP8 scales {"b{l}.fp8_sx": .., "b{l}.fp8_sh": .., ...} from
+        the MLP ranges recorded since the last reset (record_mlp_amax=True)."""
+        n = ctypes.c_int32()
+        _check(self._lib.fd_mlp_fp8_scales(self.h, None, 0, ctypes.byref(n)), "fd_mlp_fp8_scales")
+        out = (ctypes.c_float * n.value)()
+        _check(self._lib.fd_mlp_fp8_scales(self.h, out, n.value, ctypes.byref(n)),
+               "fd_mlp_fp8_scales")
+        res = {}
+        for i, p in enumerate(self._prefixes):
+            res[p + "fp8_sx"], res[p + "fp8_sh"] = float(out[2 * i]), float(out[2 * i + 1])
+        return res
 
     def kernel_ms(self) -> List[Tuple[str, float]]:
         """(kind, ms) of every timed kernel of the last frame (kernel_timing 1 or 2)."""

@@ -103,6 +103,23 @@ def test_create_rejects_bad_configs_before_touching_the_device():
         setattr(c, field, value)
         s, _ = _create(c)
         assert s == code, (field, value, s, lib.fd_last_error())
+    # FP8 MLP fields
+    bf = base.replace(dtype="bf16", head_dim=64, n_heads=2, n_kv_heads=2, d_model=128)
+    for cfg, field, value, code in [
+            (bf, "mlp_fp8", 2, fdb.FD_ERR_INVALID_ARG),
+            (bf, "record_mlp_amax", 2, fdb.FD_ERR_INVALID_ARG),
+            (base, "mlp_fp8", 1, fdb.FD_ERR_UNSUPPORTED),                  # fp32 config
+            (bf.replace(d_model=192, n_heads=3, n_kv_heads=3), "mlp_fp8", 1,
+             fdb.FD_ERR_UNSUPPORTED)]:                                      # D % 128
+        c = fdb.make_config(cfg)
+        setattr(c, field, value)
+        s, _ = _create(c)
+        assert s == code, (field, value, s, lib.fd_last_error())
+    c = fdb.make_config(bf.replace(mlp_fp8=1), record_mlp_amax=True)
+    assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
+    # FP8 without scale pointers: rejected before any device work
+    c = fdb.make_config(bf.replace(mlp_fp8=1))
+    assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     # valid shape but null weights
     s, _ = _create(fdb.make_config(base))
     assert s == fdb.FD_ERR_INVALID_ARG
@@ -120,6 +137,9 @@ def test_bad_handle_calls():
     assert lib.fd_device_bytes(None, ctypes.byref(b)) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_cache_bytes(None, ctypes.byref(b)) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_debug_read_slot(None, 0, 0, 0, None) == fdb.FD_ERR_BAD_HANDLE
+    n = ctypes.c_int32()
+    assert lib.fd_mlp_fp8_scales(None, None, 0, ctypes.byref(n)) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_block_mlp(None, 0, None, None) == fdb.FD_ERR_BAD_HANDLE
     # a pointer to memory that is not a handle (magic check)
     junk = (ctypes.c_uint32 * 64)()
     assert lib.fd_reset(ctypes.cast(junk, ctypes.c_void_p), None) == fdb.FD_ERR_BAD_HANDLE

@@ -1,0 +1,160 @@
+"""FP8 MLP on the GPU ([FD] Sec. 4.6, optimization (4): static-calibrated FP8
+quantization of all MLP layers) against the oracle's FP8 decoder.
+
+The static scales come from the oracle's calibration (its own unquantized
+decoder over the same frames), never from the CUDA path. Both sides quantize
+with the same scales, round to nearest even and take each rounding decision
+on a float32 product.
+
+Sharp check (test_block_mlp_on_identical_inputs): each block's O-projection
++ MLP kernels run on a residual stream given to both sides bit-identically,
+so the E4M3 codes of the MLP input agree exactly; relative L2 of the MLP
+output <= 1e-4.
+
+End to end, the float32/bf16 arithmetic before each decision differs between
+the two sides, and E4M3 (3 fraction bits) turns such differences into
+one-step code changes: measured on the oracle alone, a 1e-4 relative
+perturbation of the latents moves its FP8 output by 1.2e-2 (small config),
+2.4e-2 (paper head) and 3.7e-2 (480p, 12 blocks) relative L2, max abs up to
+0.21, against 9e-5 without FP8. The GPU's end-to-end distance to the oracle
+is 1.1-1.7 times that. Tolerance, re-stated for FP8 configurations: output
+relative L2 <= 6e-2 and max abs <= 0.4. The GPU's FP8 result must also move
+away from its bf16 result by about as much as the oracle's FP8 result moves
+away from its unquantized one.
+
+The GPU's own calibration (record_mlp_amax on the bf16 path) is checked
+against the oracle's scales.
+"""
+import numpy as np
+import pytest
+
+import fd_synth
+import oracle
+
+from gpu_util import errors, gpu_decode, oracle_decode, small_bf16
+
+pytestmark = pytest.mark.gpu
+
+FP8_REL_L2 = 6e-2
+FP8_MAX_ABS = 0.4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from streaming_transformer_video_b200 import lib
+    lib()
+
+
+def _fp8_case(cfg, frames=None):
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg, frames=frames)
+    scales = oracle.calibrate_fp8(cfg, w, z)
+    return cfg.replace(mlp_fp8=1), {**w, **scales}, z
+
+
+def assert_fp8_close(got, ref):
+    rel, mx = errors(got, ref)
+    assert rel <= FP8_REL_L2 and mx <= FP8_MAX_ABS, \
+        f"rel L2 {rel:.3e} (<= {FP8_REL_L2}), max abs {mx:.3e} (<= {FP8_MAX_ABS})"
+    return rel, mx
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),
+    dict(n_heads=4, n_kv_heads=2),
+    dict(window=1, frames=5),
+    dict(grid_h=17, grid_w=23, frames=4),                       # 391 tokens, ragged
+    dict(d_model=512, n_heads=8, n_kv_heads=1, frames=4),       # GQA ratio 8
+    dict(d_model=1536, n_heads=24, n_kv_heads=3, n_blocks=1, window=1, frames=3),  # XL block
+    dict(head="paper", n_refine=2, window=1, frames=3),         # refinement MLPs in FP8 too
+])
+def test_small_bf16_fp8_mlp_matches_oracle(kw):
+    cfg, w, z = _fp8_case(small_bf16(**kw))
+    assert_fp8_close(gpu_decode(cfg, w, z), oracle_decode(cfg, w, z))
+
+
+@pytest.mark.parametrize("fp8", [1, 0])
+@pytest.mark.parametrize("kw", [dict(), dict(head="paper", n_refine=2, window=1)])
+def test_block_mlp_on_identical_inputs(fp8, kw):
+    # Both sides get the same float32 residual stream, so the E4M3 codes of
+    # x + b_o are identical and only the hidden activation's rounding can
+    # differ, where its float32 value lies within ~1e-6 of an E4M3 boundary.
+    from streaming_transformer_video_b200 import FlashDecoder
+    from oracle import flashdec_oracle as fo
+    cfg = small_bf16(frames=3, **kw)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    scales = oracle.calibrate_fp8(cfg, w, z)
+    cfg8, w8 = cfg.replace(mlp_fp8=fp8), {**w, **scales}
+    w64 = {k: np.asarray(v, np.float64) for k, v in w8.items()}
+    dec = FlashDecoder(cfg8, w8)
+    rng = np.random.default_rng(11)
+    prefixes = [f"b{l}." for l in range(cfg.n_blocks)]
+    if cfg.head == "paper":
+        prefixes += [f"r{l}." for l in range(cfg.n_refine)]
+    try:
+        for i, p in enumerate(prefixes):
+            # a stream in the calibrated range (max |x| about 448 s_x)
+            x = (rng.standard_normal((cfg.L_frm, cfg.d_model)) * 100 * scales[p + "fp8_sx"])
+            x = x.astype(np.float32)
+            got = dec.debug_block_mlp(i, x).astype(np.float64)
+            xp = (x.astype(np.float64) + w64[p + "bo"]).astype(np.float32).astype(np.float64)
+            ref = fo.mlp(cfg8, w64, p, xp)
+            rel = np.linalg.norm((got - xp) - ref) / np.linalg.norm(ref)
+            # FP8: float32 accumulation-order noise plus rare hidden-code flips;
+            # bf16 MLP: the bf16 copy of x (2^-9) is its A operand
+            assert rel <= (1e-4 if fp8 else 1e-2), (p, rel)
+    finally:
+        dec.close()
+
+
+def test_fp8_differs_from_bf16_as_the_oracle_says():
+    # the GPU's FP8 result moves away from its bf16 result by about as much as
+    # the oracle's FP8 result moves away from the oracle's unquantized one
+    cfg, w, z = _fp8_case(small_bf16(frames=4))
+    g8, g16 = gpu_decode(cfg, w, z), gpu_decode(cfg.replace(mlp_fp8=0), w, z)
+    o8, o16 = oracle_decode(cfg, w, z), oracle_decode(cfg.replace(mlp_fp8=0), w, z)
+    d_gpu, d_ora = errors(g8, g16)[0], errors(o8, o16)[0]
+    assert d_ora > 1e-3
+    assert 0.5 * d_ora <= d_gpu <= 2.0 * d_ora, (d_gpu, d_ora)
+
+
+def test_gpu_calibration_matches_oracle_calibration():
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder
+    for cfg in (small_bf16(frames=4), small_bf16(head="paper", n_refine=2, window=1, frames=3)):
+        w = fd_synth.make_weights(cfg)
+        z = fd_synth.make_latents(cfg)
+        ref = oracle.calibrate_fp8(cfg, w, z)
+        dec = FlashDecoder(cfg, w, record_mlp_amax=True)
+        dec.reset()
+        lat = torch.from_numpy(z).to(torch.bfloat16).cuda()
+        out = torch.empty(cfg.out_shape, dtype=torch.bfloat16, device="cuda")
+        for t in range(z.shape[0]):
+            dec.decode_frame(lat[t], out)
+        got = dec.mlp_fp8_scales()
+        # a reset starts a new calibration
+        dec.reset()
+        assert all(v == 1.0 for v in dec.mlp_fp8_scales().values())
+        dec.close()
+        assert set(got) == set(ref)
+        for k in ref:
+            assert abs(got[k] - ref[k]) <= 2e-2 * ref[k], (k, got[k], ref[k])
+
+
+def test_fp8_causality_bit_exact():
+    cfg, w, z = _fp8_case(small_bf16(frames=5))
+    base = gpu_decode(cfg, w, z)
+    pert = gpu_decode(cfg, w, fd_synth.perturb_frame(z, 3, dtype="bf16"))
+    np.testing.assert_array_equal(pert[:3], base[:3])
+    assert not np.array_equal(pert[3], base[3])
+
+
+def test_480p_full_size_fp8_frames_0_to_3_match_oracle():
+    # the full Wan2.1-shaped 480p decoder (1560 tokens, 12 blocks) with FP8 MLPs,
+    # scales calibrated by the oracle on the same four frames
+    cfg, w, z = _fp8_case(fd_synth.CONFIGS["480p_wan21"], frames=4)
+    assert_fp8_close(gpu_decode(cfg, w, z), oracle_decode(cfg, w, z))
