@@ -60,7 +60,8 @@ def describe(cfg) -> str:
     return (f"{cfg.name}: latent {cfg.latent_ch}ch {cfg.grid_h}x{cfg.grid_w}, patch {cfg.patch} "
             f"({cfg.L_frm} tokens/frame), d={cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}"
             f" / {cfg.n_kv_heads} KV groups, {cfg.n_blocks} blocks, MLP {cfg.mlp_ratio}x, "
-            f"W={cfg.window}, {head}; each latent frame -> "
+            f"W={cfg.window}, {head}{', FP8 E4M3 MLPs' if getattr(cfg, 'mlp_fp8', 0) else ''}; "
+            f"each latent frame -> "
             f"{cfg.out_ch}x{cfg.r_t}x{cfg.out_shape[2]}x{cfg.out_shape[3]} px")
 
 
@@ -297,6 +298,19 @@ def run_flashdec(args):
     weights = fd_synth.make_weights(cfg)
     n_frames = args.warmup + args.steps
     z = fd_synth.make_latents(cfg, frames=n_frames, seed=1 + rank)
+    if args.mlp_fp8:
+        # static calibration (paper Sec. 4.6): the warm-up frames through the
+        # bf16 decoder, recording each block's MLP input / hidden ranges
+        cal = FlashDecoder(cfg, weights, record_mlp_amax=True)
+        cal.reset()
+        lat_c = torch.from_numpy(z[:args.warmup]).to(td).cuda()
+        out_c = torch.empty(cfg.out_shape, dtype=td, device="cuda")
+        for t in range(args.warmup):
+            cal.decode_frame(lat_c[t], out_c)
+        weights = {**weights, **cal.mlp_fp8_scales()}
+        cal.close()
+        del lat_c, out_c
+        cfg = cfg.replace(mlp_fp8=1)
     # events only around the attention launches (the roofline kernel): an
     # event record node per kernel would cost ~1 us each inside the step
     dec = FlashDecoder(cfg, weights, kernel_timing=2)
@@ -394,7 +408,7 @@ def run_flashdec(args):
     step_tf = step_flops / (total_ms / args.steps * 1e-3) / 1e12
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.mlp_fp8:
         per_frame, detail = oracle_sample_seconds(cfg, one_block_weights(cfg, weights), z)
         cpu = {"value": cfg.r_t / per_frame, "unit": UNIT, "cores": blas_threads(),
                "kind": "oracle",
@@ -407,7 +421,8 @@ def run_flashdec(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("bf16+e4m3-mlp" if args.mlp_fp8 else "bf16") if cfg.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": describe(cfg), "latent_frame_per_step": 1,
                    "replicas": world,
@@ -454,6 +469,9 @@ def main():
     ap.add_argument("--impl", default="flashdec", choices=["flashdec", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(fd_synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mlp-fp8", action="store_true",
+                    help="FP8 E4M3 MLP GEMMs with static scales calibrated on the warm-up "
+                         "frames by a bf16 handle that records the MLP ranges")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

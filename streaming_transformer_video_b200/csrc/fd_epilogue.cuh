@@ -177,6 +177,29 @@ __device__ __forceinline__ void rms_head(float* v, const float* g, float eps) {
   for (int d = 0; d < DH; ++d) v[d] = v[d] * r * __ldg(g + d);
 }
 
+// Unpatchify / PixelShuffle scatter of 64 finished columns of token `row`:
+// 64 / P output rows of P pixels each; column (b*P + dy)*P + dx maps to pixel
+// frame b*pl_mul + pl_add, pixel row i*P+dy, pixels j*P .. j*P+P-1. The linear
+// head has b = c*r_t + tau (pl_mul 1, pl_add 0); the spatial MLP of sub-frame
+// tau has b = c (pl_mul r_t, pl_add tau). P is a template parameter so the
+// accumulator stays in registers.
+template <int P>
+__device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int col0,
+                                              const float* acc) {
+  const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
+  const size_t out_w = size_t(p.tok_w) * P;
+  const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
+#pragma unroll
+  for (int s = 0; s < 64; s += P) {
+    const int col = col0 + s;
+    const int ct = (col / (P * P)) * p.pl_mul + p.pl_add;
+    const int dy = (col / P) % P;
+    const size_t off = size_t(ct) * plane + (size_t(i) * P + dy) * out_w + size_t(j) * P;
+    if (p.out_bf16) store_vec<bf16, P>(static_cast<bf16*>(p.out) + off, acc + s);
+    else store_vec<float, P>(static_cast<float*>(p.out) + off, acc + s);
+  }
+}
+
 // acc[64]: columns col0 .. col0+63 of token `row` (row < M guaranteed).
 template <int KIND, typename T, int DH>
 __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0, float* acc,
@@ -266,29 +289,8 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
   } else {  // EPI_FINAL
 #pragma unroll
     for (int c = 0; c < 64; ++c) acc[c] = acc[c] * rs + __ldg(p.bias + col0 + c);
-    const int P = p.P;
-    const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
-    const size_t out_w = size_t(p.tok_w) * P;
-    const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
-    // 64 columns = 64/P output rows of P pixels each; column (b*P + dy)*P + dx
-    // maps to pixel frame b*pl_mul + pl_add, pixel row i*P+dy. The linear head
-    // has b = c*r_t + tau (pl_mul 1, pl_add 0); the spatial MLP of sub-frame
-    // tau has b = c (pl_mul r_t, pl_add tau).
-    for (int s = 0; s < 64; s += P) {
-      const int col = col0 + s;
-      const int ct = (col / (P * P)) * p.pl_mul + p.pl_add;
-      const int dy = (col / P) % P;
-      const size_t off = size_t(ct) * plane + (size_t(i) * P + dy) * out_w + size_t(j) * P;
-      if (p.out_bf16) {
-        bf16* dst = static_cast<bf16*>(p.out) + off;
-        if (P == 16) store_vec<bf16, 16>(dst, acc + s);
-        else store_vec<bf16, 8>(dst, acc + s);
-      } else {
-        float* dst = static_cast<float*>(p.out) + off;
-        if (P == 16) store_vec<float, 16>(dst, acc + s);
-        else store_vec<float, 8>(dst, acc + s);
-      }
-    }
+    if (p.P == 16) pixel_scatter<16>(p, row, col0, acc);
+    else pixel_scatter<8>(p, row, col0, acc);
   }
 }
 
