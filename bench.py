@@ -54,10 +54,11 @@ def is_paper(cfg) -> bool:
 
 
 def describe(cfg) -> str:
+    streams = f"{cfg.batch} video streams per step, " if getattr(cfg, "batch", 1) > 1 else ""
     head = (f"paper head (upsample x{cfg.r_t}, {cfg.n_refine} refinement blocks over "
             f"{cfg.r_t * (cfg.window + 1)} sub-frames, spatial MLP)" if is_paper(cfg)
             else "linear head")
-    return (f"{cfg.name}: latent {cfg.latent_ch}ch {cfg.grid_h}x{cfg.grid_w}, patch {cfg.patch} "
+    return (f"{cfg.name}: {streams}latent {cfg.latent_ch}ch {cfg.grid_h}x{cfg.grid_w}, patch {cfg.patch} "
             f"({cfg.L_frm} tokens/frame), d={cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}"
             f" / {cfg.n_kv_heads} KV groups, {cfg.n_blocks} blocks, MLP {cfg.mlp_ratio}x, "
             f"W={cfg.window}, {head}{', FP8 E4M3 MLPs' if getattr(cfg, 'mlp_fp8', 0) else ''}; "
@@ -69,16 +70,16 @@ def attn_flops_per_launch(cfg):
     """FLOPs of each attention launch of one steady-state frame, in launch
     order: the backbone blocks (window of W+1 frames), then with the paper
     head r_t x n_refine refinement launches (window of r_t (W+1) sub-frames)."""
-    L, hd = cfg.L_frm, cfg.n_heads * cfg.head_dim
-    out = [4 * L * ((cfg.window + 1) * L) * hd] * cfg.n_blocks
+    L, hd, B = cfg.L_frm, cfg.n_heads * cfg.head_dim, getattr(cfg, "batch", 1)
+    out = [B * 4 * L * ((cfg.window + 1) * L) * hd] * cfg.n_blocks
     if is_paper(cfg):
-        out += [4 * L * (cfg.r_t * (cfg.window + 1) * L) * hd] * (cfg.r_t * cfg.n_refine)
+        out += [B * 4 * L * (cfg.r_t * (cfg.window + 1) * L) * hd] * (cfg.r_t * cfg.n_refine)
     return out
 
 
 def kind_flops(cfg):
-    """FLOPs of one launch of each GEMM kind (2 per MAC)."""
-    L, D = cfg.L_frm, cfg.d_model
+    """FLOPs of one launch of each GEMM kind (2 per MAC), all B streams."""
+    L, D = cfg.L_frm * getattr(cfg, "batch", 1), cfg.d_model
     f = {"qkv": 2 * L * D * cfg.qkv_dim, "oproj": 2 * L * cfg.n_heads * cfg.head_dim * D,
          "mlp_up": 2 * L * D * cfg.d_ff, "mlp_down": 2 * L * D * cfg.d_ff,
          "embed": 2 * L * cfg.c_in * D}
@@ -197,9 +198,10 @@ def sum_over_ranks(dist, v):
     return v if dist is None else _reduce(dist, v, dist.ReduceOp.SUM)
 
 
-def replica_throughput(r_t, frames_all_ranks, max_ms):
-    """Whole-job pixel frames per second of N independent decoders."""
-    return r_t * frames_all_ranks / (max_ms / 1e3)
+def replica_throughput(r_t, frames_all_ranks, max_ms, batch=1):
+    """Whole-job pixel frames per second of N independent decoders, each
+    decoding `batch` video streams per step."""
+    return r_t * batch * frames_all_ranks / (max_ms / 1e3)
 
 
 # ------------------------------------------------------------------ oracle
@@ -293,18 +295,22 @@ def run_flashdec(args):
     from streaming_transformer_video_b200 import FlashDecoder
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
-    cfg = fd_synth.CONFIGS[args.config]
+    cfg = fd_synth.CONFIGS[args.config].replace(batch=args.batch)
     td = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     weights = fd_synth.make_weights(cfg)
     n_frames = args.warmup + args.steps
-    z = fd_synth.make_latents(cfg, frames=n_frames, seed=1 + rank)
+    B = cfg.batch
+    # [T][B][C'][H'][W']: one video per stream, seeded per rank and stream
+    z = np.stack([fd_synth.make_latents(cfg, frames=n_frames, seed=1 + rank * B + b)
+                  for b in range(B)], axis=1)
+    out_shape = (B,) + tuple(cfg.out_shape)
     if args.mlp_fp8:
         # static calibration (paper Sec. 4.6): the warm-up frames through the
         # bf16 decoder, recording each block's MLP input / hidden ranges
         cal = FlashDecoder(cfg, weights, record_mlp_amax=True)
         cal.reset()
         lat_c = torch.from_numpy(z[:args.warmup]).to(td).cuda()
-        out_c = torch.empty(cfg.out_shape, dtype=td, device="cuda")
+        out_c = torch.empty(out_shape, dtype=td, device="cuda")
         for t in range(args.warmup):
             cal.decode_frame(lat_c[t], out_c)
         weights = {**weights, **cal.mlp_fp8_scales()}
@@ -316,7 +322,7 @@ def run_flashdec(args):
     dec = FlashDecoder(cfg, weights, kernel_timing=2)
     stream = torch.cuda.Stream()
     lat = torch.from_numpy(z).to(td).cuda()
-    outs = [torch.empty(cfg.out_shape, dtype=td, device="cuda") for _ in range(2)]
+    outs = [torch.empty(out_shape, dtype=td, device="cuda") for _ in range(2)]
     with torch.cuda.stream(stream):
         dec.reset(stream)
         for t in range(args.warmup):
@@ -353,12 +359,12 @@ def run_flashdec(args):
     total_ms = max_over_ranks(dist, total_ms)
     lat_ms = [a.elapsed_time(b) for a, b in ev]
     frames_all = sum_over_ranks(dist, args.steps)
-    value = replica_throughput(cfg.r_t, frames_all, total_ms)
+    value = replica_throughput(cfg.r_t, frames_all, total_ms, cfg.batch)
     launches = kernels_per_frame(cfg)
 
     # ---- end to end: host buffers through fd_decode_frame_host
     lat_h = [torch.from_numpy(z[t]).to(td).pin_memory() for t in range(n_frames)]
-    out_h = torch.empty(cfg.out_shape, dtype=td).pin_memory()
+    out_h = torch.empty(out_shape, dtype=td).pin_memory()
     e2e_steps = args.steps
     dec2 = FlashDecoder(cfg, weights)
     with torch.cuda.stream(stream):
@@ -378,9 +384,9 @@ def run_flashdec(args):
     barrier(dist)
     assert dec2.status() == 0
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1))
-    e2e_value = cfg.r_t * sum_over_ranks(dist, e2e_steps) / (e2e_ms / 1e3)
-    h2d = int(np.prod(z.shape[1:])) * (2 if td == torch.bfloat16 else 4)
-    d2h = int(np.prod(cfg.out_shape)) * (2 if td == torch.bfloat16 else 4)
+    e2e_value = cfg.r_t * cfg.batch * sum_over_ranks(dist, e2e_steps) / (e2e_ms / 1e3)
+    h2d = int(np.prod(lat.shape[1:])) * (2 if td == torch.bfloat16 else 4)
+    d2h = int(np.prod(outs[0].shape)) * (2 if td == torch.bfloat16 else 4)
     dev_bytes = dec.device_bytes()
     dec2.close()
 
@@ -409,7 +415,9 @@ def run_flashdec(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.mlp_fp8:
-        per_frame, detail = oracle_sample_seconds(cfg, one_block_weights(cfg, weights), z)
+        # the oracle decodes one stream at a time: stream 0's video
+        per_frame, detail = oracle_sample_seconds(cfg.replace(batch=1),
+                                                  one_block_weights(cfg, weights), z[:, 0])
         cpu = {"value": cfg.r_t / per_frame, "unit": UNIT, "cores": blas_threads(),
                "kind": "oracle",
                "sample": (f"frame {cfg.window + 1} (full {cfg.window + 1}-frame window) of the "
@@ -425,7 +433,7 @@ def run_flashdec(args):
         "dtype": ("bf16+e4m3-mlp" if args.mlp_fp8 else "bf16") if cfg.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {"workload": describe(cfg), "latent_frame_per_step": 1,
-                   "replicas": world,
+                   "streams_per_gpu": cfg.batch, "replicas": world,
                    "l2": "no flush: every step streams ~%.1f GB (weights + ring cache) > 126 MB L2"
                          % (dev_bytes / 1e9)},
         "p50_ms": float(np.percentile(lat_ms, 50)), "p99_ms": float(np.percentile(lat_ms, 99)),
@@ -469,6 +477,8 @@ def main():
     ap.add_argument("--impl", default="flashdec", choices=["flashdec", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(fd_synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=1,
+                    help="video streams decoded together per step (each its own video)")
     ap.add_argument("--mlp-fp8", action="store_true",
                     help="FP8 E4M3 MLP GEMMs with static scales calibrated on the warm-up "
                          "frames by a bf16 handle that records the MLP ranges")

@@ -63,6 +63,8 @@ class FDConfig:
     # 1: the MLP sublayer of every Transformer block runs on FP8 E4M3 operands
     # with static per-tensor scales (paper Sec. 4.6); bf16 configurations only
     mlp_fp8: int = 0
+    # video streams decoded together per step (each its own video and cache)
+    batch: int = 1
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property

@@ -101,6 +101,10 @@ typedef struct {
                             per block, max |x| entering the MLP and max |GELU
                             output| since the last fd_reset; read them as
                             static scales with fd_mlp_fp8_scales             */
+  int32_t batch;         /* B video streams decoded together (1 .. 64): every
+                            call takes one latent frame of each stream; each
+                            stream has its own frame counter and ring slots
+                            ([FD] Eq. 1 carries a batch dimension B)          */
 } fd_config;
 
 /*
@@ -159,16 +163,25 @@ FD_API fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd
 /*
  * Start a new video: frame counter := 0 and every ring slot zeroed, enqueued
  * on `stream` (a cudaStream_t; NULL = legacy default stream). Sec. 3.3: the
- * cache only ever holds frames of the current video.
+ * cache only ever holds frames of the current video. With batch > 1 this
+ * resets every stream.
  */
 FD_API fd_status_t fd_reset(fd_handle* h, void* stream);
 
 /*
+ * Start a new video in stream b (0 <= b < batch) only: its frame counter :=
+ * 0, enqueued on `stream`; the other streams continue. Its ring slots are not
+ * cleared: a stream at frame t only ever reads the slots of its frames
+ * max(0, t-W) .. t, all written after the reset.
+ */
+FD_API fd_status_t fd_reset_stream(fd_handle* h, int b, void* stream);
+
+/*
  * Decode the next latent frame ([FD] Sec. 3.3, steps (1)-(3), then the output
  * projection): enqueue one replay of the per-frame CUDA graph on `stream`.
- *   latent_frame: DEVICE pointer, [C'][H'][W'] contiguous, io_dtype, one frame
- *                 of a batch-1 NCTHW latent.
- *   out_pixels:   DEVICE pointer, [C][r_t][H'P/p][W'P/p] contiguous, io_dtype.
+ *   latent_frame: DEVICE pointer, [B][C'][H'][W'] contiguous, io_dtype: the
+ *                 next frame of each of the B = batch streams.
+ *   out_pixels:   DEVICE pointer, [B][C][r_t][H'P/p][W'P/p] contiguous, io_dtype.
  * Both are owned by the caller, must be 16-byte aligned and must stay valid
  * until the work on `stream` completes. Returns before the work finishes.
  * Frames must be fed strictly in order. Device-side failures are reported
@@ -203,8 +216,11 @@ FD_API const char* fd_error_string(fd_status_t s);
 /* Message of the last failure on the calling thread ("" if none). */
 FD_API const char* fd_last_error(void);
 
-/* Number of frames decoded since the last reset (synchronises). */
+/* Number of frames decoded since the last reset (synchronises); stream 0. */
 FD_API fd_status_t fd_frame_index(fd_handle* h, int64_t* t_out);
+
+/* Same for stream b (0 <= b < batch). */
+FD_API fd_status_t fd_stream_frame_index(fd_handle* h, int b, int64_t* t_out);
 
 /* Device bytes held by the handle (weights, ring cache, scratch, staging). */
 FD_API fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out);
@@ -214,8 +230,8 @@ FD_API fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out);
 FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 
 /*
- * Test/debug: copy ring slot `slot` of backbone block `block` to host memory
- * as fp32 [G][L_frm][D_h]. kv = 0 reads keys (stored after KV-norm and RoPE
+ * Test/debug: copy ring slot `slot` of backbone block `block` of stream 0 to
+ * host memory as fp32 [G][L_frm][D_h]. kv = 0 reads keys (stored after KV-norm and RoPE
  * at the frame's absolute index), kv = 1 reads values (after KV-norm).
  * Synchronous.
  */
@@ -223,11 +239,11 @@ FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv,
 
 /*
  * Test/debug: run the second half of block `block` (backbone blocks first,
- * then refinement blocks) once on a given residual stream: x_host [L_frm][D]
- * fp32 becomes the stream, the attention output is set to zero, and the
+ * then refinement blocks) once on a given residual stream: x_host becomes
+ * the stream, the attention output is set to zero, and the
  * block's O-projection (so x + b_o), MLP-up and MLP-down kernels run with
  * the handle's weights (FP8 with mlp_fp8); the resulting stream
- * x + b_o + MLP(x + b_o) is copied to out_host [L_frm][D] fp32. Both sides of
+ * x + b_o + MLP(x + b_o) is copied to out_host. Both are [batch L_frm][D] fp32. Both sides of
  * a parity test then quantize identical float32 inputs. Synchronous;
  * overwrites the handle's per-frame scratch (not the ring cache), so it must
  * not overlap a decode; records no calibration ranges.

@@ -160,17 +160,17 @@ struct KernelLaunch {
 // Where one Transformer block reads and writes: its residual stream (one
 // latent frame, or one sub-frame of the paper head) and its ring cache.
 struct BlockIO {
-  float* x32;               // [L][D] fp32 residual stream
-  void* xb;                 // [L][D] storage-type copy (A operand)
-  float* ssq;               // [L][D/32] sums of squares of x32
+  float* x32;               // [M][D] fp32 residual stream (M = B L rows)
+  void* xb;                 // [M][D] storage-type copy (A operand)
+  float* ssq;               // [M][D/32] sums of squares of x32
   const CUtensorMap* tm_x;  // map of xb (bf16 path)
-  void* kc;                 // ring keys   [layers][G][kv_rows][Dh]
-  void* vtc;                // ring values [layers][G][Dh][vt_pitch]
+  void* kc;                 // ring keys   [layers][B][G][kv_rows][Dh]
+  void* vtc;                // ring values [layers][B][G][Dh][vt_pitch]
   int kv_rows, vt_pitch;
   const CUtensorMap* tm_k;  // maps over all layers of kc / vtc (bf16 path)
   const CUtensorMap* tm_v;
   int layer;                // this block's layer inside kc / vtc
-  const FrameState* fs;     // frame state of the streamed (sub-)frame
+  const FrameState* fs;     // stream 0's state of the (sub-)frame; stride fs_stride
 };
 
 // A kernel node that writes the caller's pixel buffer (patched per call).
@@ -194,6 +194,8 @@ struct fd_handle {
   int paper = 0;                    // 1: the paper's output head
   int fp8 = 0;                      // 1: FP8 E4M3 MLP GEMMs
   int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
+  int B = 1, M = 0;                 // video streams; GEMM rows M = B L
+  int fs_stride = 1;                // FrameStates per stream: 1 (+ r_t, paper head)
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
   int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
   size_t k_bytes = 0, v_bytes = 0, rk_bytes = 0, rv_bytes = 0;
@@ -218,8 +220,8 @@ struct fd_handle {
   unsigned* amax = nullptr;                 // calibration: [blocks][2] float bits
   int n_amax = 0;
   float *x32 = nullptr, *ssq = nullptr;
-  float *xs32 = nullptr, *xss = nullptr;    // [r_t][L][D], [r_t][L][D/32]
-  void* xsb = nullptr;                      // [r_t][L][D] storage type
+  float *xs32 = nullptr, *xss = nullptr;    // [r_t][M][D], [r_t][M][D/32]
+  void* xsb = nullptr;                      // [r_t][M][D] storage type
   void *xb = nullptr, *q = nullptr, *o = nullptr, *hb = nullptr;
   float2 *rope_row = nullptr, *rope_col = nullptr;
   long long* ctr = nullptr;
@@ -402,7 +404,10 @@ const void* simt_gemm_fn(int dh) {
 
 EpiParams fd_handle::base_epi(const BlockIO& io) const {
   EpiParams e{};
-  e.M = L;
+  e.M = M;
+  e.L = L;
+  e.fs_stride = fs_stride;
+  e.out_stride = out_elems;
   e.ssq = io.ssq;
   e.ssq_parts = cfg.d_model / 32;
   e.inv_d = 1.f / float(cfg.d_model);
@@ -437,7 +442,7 @@ BlockIO fd_handle::backbone_io(int layer) {
 }
 
 BlockIO fd_handle::subframe_io(int tau, int layer) {
-  const size_t rows = size_t(tau) * L;
+  const size_t rows = size_t(tau) * M;
   const int D = cfg.d_model;
   return BlockIO{xs32 + rows * D, static_cast<char*>(xsb) + rows * D * elt,
                  xss + rows * (D / 32), bf ? &tm_xs[tau] : &tm_xb, rkc, rvtc, rkv_rows,
@@ -454,15 +459,15 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
   if (bf) {
     int bn = 0;
     if (f8) {                     // FP8 MLP: the two MLP GEMMs
-      if (kind == EPI_GELU_Q) FD_TRY((tc_gemm_pick<EPI_GELU_Q, true>(L, N, num_sms, &bn, &k)));
-      else FD_TRY((tc_gemm_pick<EPI_RESID, true>(L, N, num_sms, &bn, &k)));
+      if (kind == EPI_GELU_Q) FD_TRY((tc_gemm_pick<EPI_GELU_Q, true>(M, N, num_sms, &bn, &k)));
+      else FD_TRY((tc_gemm_pick<EPI_RESID, true>(M, N, num_sms, &bn, &k)));
     } else switch (kind) {
-      case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(L, N, num_sms, &bn, &k)); break;
-      case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(L, N, num_sms, &bn, &k)); break;
-      case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(L, N, num_sms, &bn, &k)); break;
-      case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(L, N, num_sms, &bn, &k)); break;
-      case EPI_RESID_Q: FD_TRY(tc_gemm_pick<EPI_RESID_Q>(L, N, num_sms, &bn, &k)); break;
-      default: FD_TRY(tc_gemm_pick<EPI_FINAL>(L, N, num_sms, &bn, &k)); break;
+      case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(M, N, num_sms, &bn, &k)); break;
+      case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(M, N, num_sms, &bn, &k)); break;
+      case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(M, N, num_sms, &bn, &k)); break;
+      case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(M, N, num_sms, &bn, &k)); break;
+      case EPI_RESID_Q: FD_TRY(tc_gemm_pick<EPI_RESID_Q>(M, N, num_sms, &bn, &k)); break;
+      default: FD_TRY(tc_gemm_pick<EPI_FINAL>(M, N, num_sms, &bn, &k)); break;
     }
     CUtensorMap a = tmA, b = tmB;
     int kk = K;
@@ -478,7 +483,7 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
     case EPI_UP: k.func = simt_gemm_fn<EPI_UP>(cfg.head_dim); break;
     default: k.func = simt_gemm_fn<EPI_FINAL>(cfg.head_dim); break;
   }
-  k.grid = dim3((L + 127) / 128, N / 64);
+  k.grid = dim3((M + 127) / 128, N / 64);
   k.block = dim3(128);
   k.smem = 0;
   k.kind = fd_kind;
@@ -507,8 +512,8 @@ fd_status_t fd_handle::add_out_gemm(OutNode on, int N) {
 // (+residual).
 fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
   const int D = cfg.d_model, H = cfg.n_heads, G = cfg.n_kv_heads, Dh = cfg.head_dim;
-  void* kc_l = static_cast<char*>(io.kc) + size_t(io.layer) * G * io.kv_rows * Dh * elt;
-  void* vtc_l = static_cast<char*>(io.vtc) + size_t(io.layer) * G * Dh * io.vt_pitch * elt;
+  void* kc_l = static_cast<char*>(io.kc) + size_t(io.layer) * B * G * io.kv_rows * Dh * elt;
+  void* vtc_l = static_cast<char*>(io.vtc) + size_t(io.layer) * B * G * Dh * io.vt_pitch * elt;
   // QKV + KV-norm + RoPE + ring write
   EpiParams e = base_epi(io);
   e.bias = bqkv[wi];
@@ -525,6 +530,8 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.L = L;
     ap.H = H;
     ap.G = G;
+    ap.B = B;
+    ap.fs_stride = fs_stride;
     ap.layer = io.layer;
     ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
     ap.fs = io.fs;
@@ -534,7 +541,7 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     using A = TcAttnSmem<1>;
     const void* f = reinterpret_cast<const void*>(&tc_attn_kernel<1>);
     FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
-    KernelLaunch k{f, dim3((L + 127) / 128, H), dim3(A::kThreads), size_t(A::kAlloc), FD_K_ATTN};
+    KernelLaunch k{f, dim3((L + 127) / 128, H, B), dim3(A::kThreads), size_t(A::kAlloc), FD_K_ATTN};
     CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;
     void* args[] = {&a, &b, &c, &ap};
     FD_TRY(add_kernel(k, args));
@@ -549,12 +556,14 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.G = G;
     ap.kv_rows = io.kv_rows;
     ap.vt_pitch = io.vt_pitch;
+    ap.B = B;
+    ap.fs_stride = fs_stride;
     ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
     ap.fs = io.fs;
     ap.status = status;
     const void* f = Dh == 32 ? reinterpret_cast<const void*>(&simt_attn_kernel<32>)
                              : reinterpret_cast<const void*>(&simt_attn_kernel<64>);
-    KernelLaunch k{f, dim3((L + 63) / 64, H), dim3(64), 0, FD_K_ATTN};
+    KernelLaunch k{f, dim3((L + 63) / 64, H, B), dim3(64), 0, FD_K_ATTN};
     void* args[] = {&ap};
     FD_TRY(add_kernel(k, args));
   }
@@ -619,9 +628,9 @@ fd_status_t fd_handle::build_graph() {
                    FD_K_STEP_BEGIN};
     long long* c = ctr;
     FrameState* f = fs;
-    int W = cfg.window, dh = cfg.head_dim, n_sub = paper ? cfg.r_t : 0;
+    int W = cfg.window, dh = cfg.head_dim, n_sub = paper ? cfg.r_t : 0, nb = B;
     float th = cfg.rope_theta;
-    void* args[] = {&c, &f, &W, &dh, &th, &n_sub};
+    void* args[] = {&c, &f, &W, &dh, &th, &n_sub, &nb};
     FD_TRY(add_kernel(k, args));
   }
   // embed
@@ -634,6 +643,7 @@ fd_status_t fd_handle::build_graph() {
     embed_p.p = cfg.patch;
     embed_p.tok_w = tok_w;
     embed_p.L = L;
+    embed_p.M = M;
     embed_p.c_in = c_in;
     embed_p.wT = embed_wT;
     embed_p.b = embed_b;
@@ -643,7 +653,7 @@ fd_status_t fd_handle::build_graph() {
     embed_p.ssq = ssq;
     const void* f = bf ? reinterpret_cast<const void*>(&embed_kernel<bf16>)
                        : reinterpret_cast<const void*>(&embed_kernel<float>);
-    embed_launch = KernelLaunch{f, dim3((L + kEmbedTok - 1) / kEmbedTok), dim3(256),
+    embed_launch = KernelLaunch{f, dim3((M + kEmbedTok - 1) / kEmbedTok), dim3(256),
                                 size_t(kEmbedTok) * c_in * 4, FD_K_EMBED};
     void* args[] = {&embed_p};
     FD_TRY(add_kernel(embed_launch, args, &embed_node));
@@ -678,7 +688,7 @@ fd_status_t fd_handle::build_graph() {
     for (int tau = 0; tau < cfg.r_t; ++tau) {
       // refinement blocks: sub-frame t r_t + tau in the ring of r_t (W+1)
       for (int l = 0; l < cfg.n_refine; ++l) FD_TRY(add_block(cfg.n_blocks + l, subframe_io(tau, l)));
-      // spatial MLP layer 1: GELU(RMSNorm(xs) sp1_w^T + sp1_b) -> hidden [L][D]
+      // spatial MLP layer 1: GELU(RMSNorm(xs) sp1_w^T + sp1_b) -> hidden [M][D]
       const BlockIO io = subframe_io(tau, 0);
       e = base_epi(io);
       e.bias = bsp1;
@@ -750,6 +760,8 @@ fd_status_t validate(const fd_config* c) {
   if (L * (c->window + 1) > (1LL << 30))
     return fail(FD_ERR_UNSUPPORTED, "config: window of %lld tokens is too large",
                 L * (c->window + 1));
+  if (c->batch < 1 || c->batch > fd::kMaxStreams)
+    return fail(FD_ERR_INVALID_ARG, "config: batch must be 1 .. %d (got %d)", fd::kMaxStreams, c->batch);
   if (c->kernel_timing < 0 || c->kernel_timing > 2)
     return fail(FD_ERR_INVALID_ARG, "config: kernel_timing must be 0, 1 or 2");
   if (c->head_mode != 0 && c->head_mode != 1)
@@ -783,6 +795,9 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   h->tok_h = c.grid_h / c.patch;
   h->tok_w = c.grid_w / c.patch;
   h->L = h->tok_h * h->tok_w;
+  h->B = c.batch;
+  h->M = h->B * h->L;
+  h->fs_stride = 1 + (c.head_mode == 1 ? c.r_t : 0);
   h->c_in = c.latent_ch * c.patch * c.patch;
   h->qkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
   h->dff = c.mlp_ratio * c.d_model;
@@ -853,22 +868,23 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(h->upload_f32(&h->bout, w->out_b, c_px));
   }
 
-  // ---- ring caches: K [layers][G][rows][Dh], V^T [layers][G][Dh][pitch];
+  // ---- ring caches: K [layers][B][G][rows][Dh], V^T [layers][B][G][Dh][pitch];
   // backbone rows = (W+1) L, refinement rows = r_t (W+1) L
-  h->k_bytes = size_t(NB) * G * h->kv_rows * Dh * h->elt;
-  h->v_bytes = size_t(NB) * G * Dh * h->vt_pitch * h->elt;
+  const int BG = h->B * G;
+  h->k_bytes = size_t(NB) * BG * h->kv_rows * Dh * h->elt;
+  h->v_bytes = size_t(NB) * BG * Dh * h->vt_pitch * h->elt;
   FD_TRY(h->alloc(&h->kc, h->k_bytes));
   FD_TRY(h->alloc(&h->vtc, h->v_bytes));
   if (h->paper) {
-    h->rk_bytes = size_t(NR) * G * h->rkv_rows * Dh * h->elt;
-    h->rv_bytes = size_t(NR) * G * Dh * h->rvt_pitch * h->elt;
+    h->rk_bytes = size_t(NR) * BG * h->rkv_rows * Dh * h->elt;
+    h->rv_bytes = size_t(NR) * BG * Dh * h->rvt_pitch * h->elt;
     FD_TRY(h->alloc(&h->rkc, h->rk_bytes));
     FD_TRY(h->alloc(&h->rvtc, h->rv_bytes));
   }
   h->cache_bytes = h->k_bytes + h->v_bytes + h->rk_bytes + h->rv_bytes;
 
   // ---- scratch
-  const size_t L = h->L;
+  const size_t L = h->M;                 // every per-frame buffer holds B frames
   FD_TRY(h->alloc(&h->x32, L * D * 4));
   FD_TRY(h->alloc(&h->xb, L * D * h->elt));
   FD_TRY(h->alloc(&h->ssq, L * (D / 32) * 4));
@@ -885,11 +901,11 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     h->n_amax = 2 * (NB + NR);
     FD_TRY(h->alloc(&h->amax, size_t(h->n_amax) * 4));
   }
-  FD_TRY(h->alloc(&h->ctr, 64));
-  FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * (1 + (h->paper ? c.r_t : 0))));
+  FD_TRY(h->alloc(&h->ctr, size_t(h->B) * 8));
+  FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * h->fs_stride * h->B));
   FD_TRY(h->alloc(&h->status, 16));
-  FD_TRY(h->alloc(&h->latent_stage, round_up(h->latent_elems * h->io_elt, 256)));
-  FD_TRY(h->alloc(&h->out_stage, round_up(h->out_elems * h->io_elt, 256)));
+  FD_TRY(h->alloc(&h->latent_stage, round_up(h->B * h->latent_elems * h->io_elt, 256)));
+  FD_TRY(h->alloc(&h->out_stage, round_up(h->B * h->out_elems * h->io_elt, 256)));
 
   // ---- spatial RoPE tables (fp64 angles): row part and column part,
   // d_s = 3 D_h / 8 dims each, pair m at frequency theta^(-2m/d_s)
@@ -944,29 +960,30 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
         FD_TRY(make_tmap_2d(&m, static_cast<char*>(h->xsb) + size_t(tau) * L * D * 2, L, D, 128));
         h->tm_xs.push_back(m);
       }
-      const uint64_t kd[3] = {64, uint64_t(h->rkv_rows), uint64_t(NR) * G};
+      const uint64_t kd[3] = {64, uint64_t(h->rkv_rows), uint64_t(NR) * BG};
       const uint64_t ks[2] = {64 * 2, uint64_t(h->rkv_rows) * 64 * 2};
       const uint32_t kb[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_rk, h->rkc, 3, kd, ks, kb));
-      const uint64_t vd[3] = {uint64_t(h->rvt_pitch), 64, uint64_t(NR) * G};
+      const uint64_t vd[3] = {uint64_t(h->rvt_pitch), 64, uint64_t(NR) * BG};
       const uint64_t vs[2] = {uint64_t(h->rvt_pitch) * 2, uint64_t(h->rvt_pitch) * 64 * 2};
       const uint32_t vb[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_rv, h->rvtc, 3, vd, vs, vb));
     }
-    {   // Q [H][L][64]: box 64 x 128 x 1
-      const uint64_t dims[3] = {64, L, uint64_t(H)};
-      const uint64_t str[2] = {64 * 2, L * 64 * 2};
-      const uint32_t box[3] = {64, 128, 1};
-      FD_TRY(make_tmap(&h->tm_q, h->q, 3, dims, str, box));
+    {   // Q [H][B][L_frm][64]: box 64 x 128 x 1 x 1; a stream's last tile reads zeros
+      const uint64_t Lf = uint64_t(h->L);
+      const uint64_t dims[4] = {64, Lf, uint64_t(h->B), uint64_t(H)};
+      const uint64_t str[3] = {64 * 2, Lf * 64 * 2, uint64_t(h->B) * Lf * 64 * 2};
+      const uint32_t box[4] = {64, 128, 1, 1};
+      FD_TRY(make_tmap(&h->tm_q, h->q, 4, dims, str, box));
     }
     {   // K [NB*G][kv_rows][64]: box 64 dims x 64 keys x 1
-      const uint64_t dims[3] = {64, uint64_t(h->kv_rows), uint64_t(NB) * G};
+      const uint64_t dims[3] = {64, uint64_t(h->kv_rows), uint64_t(NB) * BG};
       const uint64_t str[2] = {64 * 2, uint64_t(h->kv_rows) * 64 * 2};
       const uint32_t box[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_k, h->kc, 3, dims, str, box));
     }
     {   // V^T [NB*G][64][vt_pitch]: box 64 keys x 64 dims x 1
-      const uint64_t dims[3] = {uint64_t(h->vt_pitch), 64, uint64_t(NB) * G};
+      const uint64_t dims[3] = {uint64_t(h->vt_pitch), 64, uint64_t(NB) * BG};
       const uint64_t str[2] = {uint64_t(h->vt_pitch) * 2, uint64_t(h->vt_pitch) * 64 * 2};
       const uint32_t box[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_v, h->vtc, 3, dims, str, box));
@@ -980,7 +997,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_CUDA(cudaMemset(h->rkc, 0, h->rk_bytes));
     FD_CUDA(cudaMemset(h->rvtc, 0, h->rv_bytes));
   }
-  FD_CUDA(cudaMemset(h->ctr, 0, 64));
+  FD_CUDA(cudaMemset(h->ctr, 0, size_t(h->B) * 8));
   FD_CUDA(cudaMemset(h->status, 0, 16));
   if (h->amax) FD_CUDA(cudaMemset(h->amax, 0, size_t(h->n_amax) * 4));
   FD_CUDA(cudaMemset(h->fs, 0, sizeof(FrameState)));
@@ -1081,10 +1098,30 @@ fd_status_t fd_reset(fd_handle* h, void* stream) {
     FD_CUDA(cudaMemsetAsync(h->rkc, 0, h->rk_bytes, s));
     FD_CUDA(cudaMemsetAsync(h->rvtc, 0, h->rv_bytes, s));
   }
-  FD_CUDA(cudaMemsetAsync(h->ctr, 0, 64, s));
+  FD_CUDA(cudaMemsetAsync(h->ctr, 0, size_t(h->B) * 8, s));
   FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
   if (h->amax) FD_CUDA(cudaMemsetAsync(h->amax, 0, size_t(h->n_amax) * 4, s));
   h->last_stream = s;
+  return FD_OK;
+}
+
+fd_status_t fd_reset_stream(fd_handle* h, int b, void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_reset_stream: invalid handle");
+  if (b < 0 || b >= h->B) return fail(FD_ERR_INVALID_ARG, "fd_reset_stream: stream %d out of range", b);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_CUDA(cudaMemsetAsync(h->ctr + b, 0, 8, s));
+  h->last_stream = s;
+  return FD_OK;
+}
+
+fd_status_t fd_stream_frame_index(fd_handle* h, int b, int64_t* t_out) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_stream_frame_index: invalid handle");
+  if (b < 0 || b >= h->B || !t_out)
+    return fail(FD_ERR_INVALID_ARG, "fd_stream_frame_index: bad stream or null output");
+  FD_CUDA(cudaStreamSynchronize(h->last_stream));
+  long long t = 0;
+  FD_CUDA(cudaMemcpy(&t, h->ctr + b, 8, cudaMemcpyDeviceToHost));
+  *t_out = t;
   return FD_OK;
 }
 
@@ -1112,11 +1149,11 @@ fd_status_t fd_decode_frame_host(fd_handle* h, const void* latent_host, void* ou
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame_host: invalid handle");
   if (!latent_host || !out_host) return fail(FD_ERR_INVALID_ARG, "fd_decode_frame_host: null buffer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  FD_CUDA(cudaMemcpyAsync(h->latent_stage, latent_host, h->latent_elems * h->io_elt,
+  FD_CUDA(cudaMemcpyAsync(h->latent_stage, latent_host, h->B * h->latent_elems * h->io_elt,
                           cudaMemcpyHostToDevice, s));
   FD_TRY(patch_io(h, h->latent_stage, h->out_stage));
   FD_CUDA(cudaGraphLaunch(h->exec, s));
-  FD_CUDA(cudaMemcpyAsync(out_host, h->out_stage, h->out_elems * h->io_elt,
+  FD_CUDA(cudaMemcpyAsync(out_host, h->out_stage, h->B * h->out_elems * h->io_elt,
                           cudaMemcpyDeviceToHost, s));
   h->last_stream = s;
   return FD_OK;
@@ -1190,7 +1227,7 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
   if (kv == 0) {
     raw.resize(n * h->elt);
     for (int g = 0; g < G; ++g) {
-      const size_t src = ((size_t(block) * G + g) * h->kv_rows + size_t(slot) * L) * Dh * h->elt;
+      const size_t src = ((size_t(block) * h->B * G + g) * h->kv_rows + size_t(slot) * L) * Dh * h->elt;
       FD_CUDA(cudaMemcpy(raw.data() + size_t(g) * L * Dh * h->elt,
                          static_cast<char*>(h->kc) + src, size_t(L) * Dh * h->elt,
                          cudaMemcpyDeviceToHost));
@@ -1203,7 +1240,7 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
     std::vector<uint8_t> rows(size_t(L) * h->elt);
     for (int g = 0; g < G; ++g)
       for (int d = 0; d < Dh; ++d) {
-        const size_t src = ((size_t(block) * G + g) * Dh + d) * h->vt_pitch + size_t(slot) * L;
+        const size_t src = ((size_t(block) * h->B * G + g) * Dh + d) * h->vt_pitch + size_t(slot) * L;
         FD_CUDA(cudaMemcpy(rows.data(), static_cast<char*>(h->vtc) + src * h->elt,
                            size_t(L) * h->elt, cudaMemcpyDeviceToHost));
         for (int n2 = 0; n2 < L; ++n2)
@@ -1222,9 +1259,9 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   if (block < 0 || block >= n_all || !x_host || !out_host)
     return fail(FD_ERR_INVALID_ARG, "fd_debug_block_mlp: bad block or null buffer");
   FD_CUDA(cudaDeviceSynchronize());
-  const size_t n = size_t(h->L) * c.d_model;
+  const size_t n = size_t(h->M) * c.d_model;
   FD_CUDA(cudaMemcpy(h->x32, x_host, n * 4, cudaMemcpyHostToDevice));
-  FD_CUDA(cudaMemset(h->o, 0, size_t(h->L) * c.n_heads * c.head_dim * h->elt));
+  FD_CUDA(cudaMemset(h->o, 0, size_t(h->M) * c.n_heads * c.head_dim * h->elt));
   // a one-off graph of the block's post-attention kernels on the backbone
   // stream; no timing events, no calibration records
   cudaGraph_t saved_graph = h->graph;

@@ -6,8 +6,10 @@
 // are always the contiguous range [0, n_valid*L) and softmax, being
 // invariant to the order of keys, needs no slot bookkeeping.
 //
-// One CTA = one head x QT query tiles of 128 (QT = 1 or 2). Keys are
-// consumed in tiles of 64; every K/V stage is shared by the QT query tiles.
+// One CTA = one head x QT query tiles of 128 (QT = 1 or 2) of one video
+// stream (blockIdx.z; each stream has its own frame state and cache slab).
+// Keys are consumed in tiles of 64; every K/V stage is shared by the QT
+// query tiles.
 // Warps:
 //   0            TMA: the Q tiles once, then per stage K (64 keys x 64) and
 //                the transposed V (64 dims x 64 keys)
@@ -31,9 +33,11 @@
 namespace fd {
 
 struct TcAttnParams {
-  void* o;            // [L][H*64] bf16
+  void* o;            // [B][L][H*64] bf16
   int L, H, G;
-  int layer;          // block index: third coordinate base of the cache maps
+  int B;              // video streams
+  int layer;          // block index: cache map slab (layer * B + stream) * G + g
+  int fs_stride;      // FrameStates per stream
   float scale_log2;   // log2(e) / sqrt(64)
   const FrameState* fs;
   int* status;
@@ -148,10 +152,10 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
   auto o_final = [&](int t) { return tb + 9 * t + 8; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (128 * QT), h = blockIdx.y;
+  const int q0 = blockIdx.x * (128 * QT), h = blockIdx.y, bs = blockIdx.z;
   const int g = h / (p.H / p.G);
-  const int lg = p.layer * p.G + g;
-  const int n_keys = p.fs->n_valid * p.L;
+  const int lg = (p.layer * p.B + bs) * p.G + g;
+  const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
   const int n_kt = (n_keys + 63) / 64;
 
   if (threadIdx.x == 0) {
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
     if (lane == 0) {                                       // ---- TMA producer
       mbar_arrive_expect_tx(q_full, QT * 16384);
       for (int t = 0; t < QT; ++t)
-        tma_load_3d(smem + S::kQ + t * 16384, &tmQ, 0, q0 + t * 128, h, q_full);
+        tma_load_4d(smem + S::kQ + t * 16384, &tmQ, 0, q0 + t * 128, bs, h, q_full);
       for (int j = 0; j < n_kt; ++j) {
         const int st = j % ST;
         if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
@@ -314,7 +318,8 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
           v[c] = __uint_as_float(o0[c]) * inv;
           v[32 + c] = __uint_as_float(o1[c]) * inv;
         }
-        store_vec<bf16, 64>(static_cast<bf16*>(p.o) + size_t(row) * p.H * 64 + size_t(h) * 64, v);
+        store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
+                                size_t(h) * 64, v);
       }
     }
   }

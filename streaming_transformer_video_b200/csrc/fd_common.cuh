@@ -17,6 +17,7 @@ typedef __nv_bfloat16 bf16;
 // Longest head the kernels support (RoPE tables are sized from it).
 constexpr int kMaxHeadDim = 64;
 constexpr int kMaxTemporalPairs = kMaxHeadDim / 8;   // D_h/4 dims -> D_h/8 pairs
+constexpr int kMaxStreams = 64;                      // video streams per handle
 
 // Per-frame state, written once per frame by the step_begin kernel from the
 // device frame counter and read by every later kernel of the frame.

@@ -44,7 +44,8 @@ constexpr bool epi_normed(int kind) {
 }
 
 struct EpiParams {
-  int M;                 // rows (tokens of the frame)
+  int M;                 // rows: B video streams x L tokens, row = b L + n
+  int L;                 // tokens per frame of one stream
   int N;                 // GEMM output columns
   const float* bias;     // [N]
   // RMSNorm row scale (QKV, GELU, FINAL; none when ssq is null)
@@ -59,22 +60,24 @@ struct EpiParams {
   int D;
   // QKV
   void* q;               // [H][M][Dh]
-  void* kc;              // this block's keys   [G][kv_rows][Dh]
-  void* vtc;             // this block's values [G][Dh][vt_pitch] (transposed)
+  void* kc;              // this block's keys   [B][G][kv_rows][Dh]
+  void* vtc;             // this block's values [B][G][Dh][vt_pitch] (transposed)
   int H, G, Dh;
   int kv_rows;           // (W+1) * M
   int vt_pitch;          // row pitch of the transposed values (elements)
   const float* gk;       // [Dh] KV-norm gains
   const float* gv;
   int kv_norm;
-  const FrameState* fs;
+  const FrameState* fs;  // stream b's state: fs[b * fs_stride]
+  int fs_stride;
   const float2* rope_row;  // [tok_h][d_s/2] (cos, sin)
   const float2* rope_col;  // [tok_w][d_s/2]
   int tok_w;
   // GELU
   void* hout;            // [M][N]
   // FINAL
-  void* out;             // [C][r_t][tok_h*P][tok_w*P]
+  void* out;             // [B][C][r_t][tok_h*P][tok_w*P]
+  size_t out_stride;     // pixels per stream
   int out_bf16;          // pixel element type
   int P;                 // pixels per token side
   int tok_h;
@@ -133,18 +136,20 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
 }
 
-// In-place 3D-RoPE of one head vector v[DH] of token `row`: pairs (2m, 2m+1)
-// of the temporal part [0, DH/4) rotate by the frame's angle, the row part
-// [DH/4, DH/4 + 3DH/8) by the token's grid row, the column part by its column.
+// In-place 3D-RoPE of one head vector v[DH] of token n of a frame with state
+// fs: pairs (2m, 2m+1) of the temporal part [0, DH/4) rotate by the frame's
+// angle, the row part [DH/4, DH/4 + 3DH/8) by the token's grid row, the
+// column part by its column.
 template <int DH>
-__device__ __forceinline__ void rope_head(float* v, int row, const EpiParams& p) {
+__device__ __forceinline__ void rope_head(float* v, int n, const FrameState* fs,
+                                          const EpiParams& p) {
   constexpr int dt = DH / 4, ds = 3 * DH / 8;
-  const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
+  const int i = n / p.tok_w, j = n - (n / p.tok_w) * p.tok_w;
   const float2* rr = p.rope_row + size_t(i) * (ds / 2);
   const float2* rc = p.rope_col + size_t(j) * (ds / 2);
 #pragma unroll
   for (int m = 0; m < dt / 2; ++m) {
-    const float2 cs = p.fs->rope_t[m];
+    const float2 cs = fs->rope_t[m];
     const float a = v[2 * m], b = v[2 * m + 1];
     v[2 * m] = a * cs.x - b * cs.y;
     v[2 * m + 1] = a * cs.y + b * cs.x;
@@ -186,7 +191,8 @@ __device__ __forceinline__ void rms_head(float* v, const float* g, float eps) {
 template <int P>
 __device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int col0,
                                               const float* acc) {
-  const int i = row / p.tok_w, j = row - (row / p.tok_w) * p.tok_w;
+  const int b = row / p.L, n = row - b * p.L;              // stream, token
+  const int i = n / p.tok_w, j = n - (n / p.tok_w) * p.tok_w;
   const size_t out_w = size_t(p.tok_w) * P;
   const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
 #pragma unroll
@@ -194,7 +200,8 @@ __device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int c
     const int col = col0 + s;
     const int ct = (col / (P * P)) * p.pl_mul + p.pl_add;
     const int dy = (col / P) % P;
-    const size_t off = size_t(ct) * plane + (size_t(i) * P + dy) * out_w + size_t(j) * P;
+    const size_t off = size_t(b) * p.out_stride + size_t(ct) * plane +
+                       (size_t(i) * P + dy) * out_w + size_t(j) * P;
     if (p.out_bf16) store_vec<bf16, P>(static_cast<bf16*>(p.out) + off, acc + s);
     else store_vec<float, P>(static_cast<float*>(p.out) + off, acc + s);
   }
@@ -205,6 +212,8 @@ template <int KIND, typename T, int DH>
 __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0, float* acc,
                                            float rs) {
   if constexpr (KIND == EPI_QKV) {
+    const int b = row / p.L, n = row - b * p.L;            // stream, token
+    const FrameState* fs = p.fs + size_t(b) * p.fs_stride;
 #pragma unroll
     for (int hh = 0; hh < 64 / DH; ++hh) {
       float* v = acc + hh * DH;
@@ -213,21 +222,21 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
 #pragma unroll
       for (int d = 0; d < DH; ++d) v[d] = v[d] * rs + __ldg(p.bias + col + d);
       if (head < p.H) {                                   // query head
-        rope_head<DH>(v, row, p);
+        rope_head<DH>(v, n, fs, p);
         T* dst = static_cast<T*>(p.q) + (size_t(head) * p.M + row) * DH;
         store_vec<T, DH>(dst, v);
       } else if (head < p.H + p.G) {                      // key group
         const int g = head - p.H;
         if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
-        rope_head<DH>(v, row, p);
-        const int key = p.fs->slot * p.M + row;
-        T* dst = static_cast<T*>(p.kc) + (size_t(g) * p.kv_rows + key) * DH;
+        rope_head<DH>(v, n, fs, p);
+        const int key = fs->slot * p.L + n;
+        T* dst = static_cast<T*>(p.kc) + ((size_t(b) * p.G + g) * p.kv_rows + key) * DH;
         store_vec<T, DH>(dst, v);
       } else {                                            // value group
         const int g = head - p.H - p.G;
         if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
-        const int key = p.fs->slot * p.M + row;
-        T* dst = static_cast<T*>(p.vtc) + size_t(g) * DH * p.vt_pitch + key;
+        const int key = fs->slot * p.L + n;
+        T* dst = static_cast<T*>(p.vtc) + (size_t(b) * p.G + g) * DH * p.vt_pitch + key;
 #pragma unroll
         for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch] = from_f<T>(v[d]);
       }

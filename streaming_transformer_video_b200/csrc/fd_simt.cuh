@@ -31,22 +31,25 @@ __device__ void frame_state(FrameState* fs, long long t, int cap, int head_dim, 
   }
 }
 
-// fs[0]: latent frame t = counter in the backbone ring of W+1 frames.
-// fs[1 + tau], tau < n_sub (paper head, n_sub = r_t): sub-frame t r_t + tau
-// in the refinement ring of r_t (W+1) sub-frames (paper Sec. 3.4, Step 2).
-// Thread tau + 1 writes sub-frame tau; the counter becomes t + 1.
+// B video streams, each with its own counter ctr[b] and 1 + n_sub states
+// fs[b (1 + n_sub) + k]:
+//   k = 0: latent frame t = ctr[b] in the backbone ring of W+1 frames;
+//   k = 1 + tau, tau < n_sub (paper head, n_sub = r_t): sub-frame t r_t + tau
+//   in the refinement ring of r_t (W+1) sub-frames (paper Sec. 3.4, Step 2).
+// Every counter then advances by one. One CTA of 32 threads.
 __global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int head_dim,
-                                  float theta, int n_sub) {
-  if (blockIdx.x != 0) return;
-  const long long t = *ctr;
-  __syncwarp();
-  const int i = threadIdx.x;
-  if (i == 0) {
-    frame_state(fs, t, W + 1, head_dim, theta);
-    *ctr = t + 1;
-  } else if (i <= n_sub) {
-    frame_state(fs + i, t * n_sub + (i - 1), n_sub * (W + 1), head_dim, theta);
+                                  float theta, int n_sub, int B) {
+  __shared__ long long t0[kMaxStreams];
+  for (int b = threadIdx.x; b < B; b += blockDim.x) t0[b] = ctr[b];
+  __syncthreads();
+  const int per = 1 + n_sub;
+  for (int i = threadIdx.x; i < B * per; i += blockDim.x) {
+    const int b = i / per, k = i - b * per;
+    if (k == 0) frame_state(fs + i, t0[b], W + 1, head_dim, theta);
+    else frame_state(fs + i, t0[b] * n_sub + (k - 1), n_sub * (W + 1), head_dim, theta);
   }
+  __syncthreads();
+  for (int b = threadIdx.x; b < B; b += blockDim.x) ctr[b] = t0[b] + 1;
 }
 
 // ---------------------------------------------------------------- self-test
@@ -67,17 +70,18 @@ __global__ void wait_timeout_selftest_kernel(int* status, unsigned long long tim
 
 // ---------------------------------------------------------------- embed
 struct EmbedParams {
-  const void* latent;     // [C'][H'][W'] io type
+  const void* latent;     // [B][C'][H'][W'] io type
   int latent_bf16;
   int C, Hl, Wl, p;       // latent channels, rows, columns, patch
-  int tok_w, L;
+  int tok_w, L;           // L tokens per frame of one stream
+  int M;                  // B L rows
   int c_in;               // C' p^2
   const float* wT;        // [c_in][D] (transposed projection)
   const float* b;         // [D]
   int D;
-  float* x32;             // [L][D]
-  void* xb;               // [L][D] storage type
-  float* ssq;             // [L][D/32]
+  float* x32;             // [M][D]
+  void* xb;               // [M][D] storage type
+  float* ssq;             // [M][D/32]
 };
 
 constexpr int kEmbedTok = 8;
@@ -93,10 +97,11 @@ __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
     const int tk = idx / p.c_in, ch = idx - tk * p.c_in;
     const int n = n0 + tk;
     float v = 0.f;
-    if (n < p.L) {
+    if (n < p.M) {
+      const int b = n / p.L, nt = n - b * p.L;             // stream, token
       const int c = ch / (p.p * p.p), dy = (ch / p.p) % p.p, dx = ch % p.p;
-      const int i = n / p.tok_w, j = n - (n / p.tok_w) * p.tok_w;
-      const size_t off = (size_t(c) * p.Hl + i * p.p + dy) * p.Wl + j * p.p + dx;
+      const int i = nt / p.tok_w, j = nt - (nt / p.tok_w) * p.tok_w;
+      const size_t off = ((size_t(b) * p.C + c) * p.Hl + i * p.p + dy) * p.Wl + j * p.p + dx;
       v = p.latent_bf16 ? __bfloat162float(static_cast<const bf16*>(p.latent)[off])
                         : static_cast<const float*>(p.latent)[off];
     }
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
       float s = acc[t] * acc[t];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (n < p.L) {
+      if (n < p.M) {
         p.x32[size_t(n) * p.D + d] = acc[t];
         static_cast<T*>(p.xb)[size_t(n) * p.D + d] = from_f<T>(acc[t]);
         if ((threadIdx.x & 31) == 0) p.ssq[size_t(n) * parts + d / 32] = s;
@@ -165,11 +170,12 @@ __global__ void __launch_bounds__(128) simt_gemm_kernel(const float* A, const fl
 
 // ---------------------------------------------------------------- simt_attn
 struct AttnParams {
-  const void* q;          // [H][L][Dh]
-  const void* kc;         // [G][kv_rows][Dh]
-  const void* vtc;        // [G][Dh][vt_pitch]
-  void* o;                // [L][H*Dh]
+  const void* q;          // [H][B][L][Dh]
+  const void* kc;         // [B][G][kv_rows][Dh]
+  const void* vtc;        // [B][G][Dh][vt_pitch]
+  void* o;                // [B][L][H*Dh]
   int L, H, G, kv_rows, vt_pitch;
+  int B, fs_stride;       // streams; FrameStates per stream
   float scale_log2;       // log2(e) / sqrt(Dh)
   const FrameState* fs;
   int* status;
@@ -181,16 +187,17 @@ template <int DH>
 __global__ void __launch_bounds__(64) simt_attn_kernel(AttnParams p) {
   __shared__ float Ks[32][DH + 1];
   __shared__ float Vs[32][DH + 1];
-  const int h = blockIdx.y, g = h / (p.H / p.G);
+  const int h = blockIdx.y, g = h / (p.H / p.G), bs = blockIdx.z;
   const int row = blockIdx.x * 64 + threadIdx.x;
-  const int n_keys = p.fs->n_valid * p.L;
-  const float* qp = static_cast<const float*>(p.q) + (size_t(h) * p.L + (row < p.L ? row : 0)) * DH;
+  const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
+  const float* qp = static_cast<const float*>(p.q) +
+                    ((size_t(h) * p.B + bs) * p.L + (row < p.L ? row : 0)) * DH;
   float q[DH], o[DH];
 #pragma unroll
   for (int d = 0; d < DH; ++d) { q[d] = qp[d] * p.scale_log2; o[d] = 0.f; }
   float m = -INFINITY, l = 0.f;
-  const float* kg = static_cast<const float*>(p.kc) + size_t(g) * p.kv_rows * DH;
-  const float* vg = static_cast<const float*>(p.vtc) + size_t(g) * DH * p.vt_pitch;
+  const float* kg = static_cast<const float*>(p.kc) + (size_t(bs) * p.G + g) * p.kv_rows * DH;
+  const float* vg = static_cast<const float*>(p.vtc) + (size_t(bs) * p.G + g) * DH * p.vt_pitch;
   for (int k0 = 0; k0 < n_keys; k0 += 32) {
     for (int idx = threadIdx.x; idx < 32 * DH; idx += 64) {
       const int j = idx / DH, d = idx % DH;
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(64) simt_attn_kernel(AttnParams p) {
   }
   if (row < p.L) {
     const float inv = 1.f / l;
-    float* op = static_cast<float*>(p.o) + size_t(row) * p.H * DH + size_t(h) * DH;
+    float* op = static_cast<float*>(p.o) + (size_t(bs) * p.L + row) * p.H * DH + size_t(h) * DH;
 #pragma unroll
     for (int d = 0; d < DH; ++d) op[d] = o[d] * inv;
   }

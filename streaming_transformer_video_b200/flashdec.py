@@ -27,7 +27,8 @@ HEAD_MODES = {"linear": 0, "paper": 1}
 EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
            "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
-           "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp"]
+           "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp",
+           "fd_reset_stream", "fd_stream_frame_index"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -38,7 +39,7 @@ class FDConfigC(ctypes.Structure):
         ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
         ("kernel_timing", ctypes.c_int32), ("head_mode", ctypes.c_int32),
         ("n_refine", ctypes.c_int32), ("mlp_fp8", ctypes.c_int32),
-        ("record_mlp_amax", ctypes.c_int32)]
+        ("record_mlp_amax", ctypes.c_int32), ("batch", ctypes.c_int32)]
 
 
 _PF = ctypes.POINTER(ctypes.c_float)
@@ -83,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_selftest_wait_timeout.argtypes = [i32]
     lib.fd_mlp_fp8_scales.argtypes = [vp, _PF, i32, ctypes.POINTER(i32)]
     lib.fd_debug_block_mlp.argtypes = [vp, i32, _PF, _PF]
+    lib.fd_reset_stream.argtypes = [vp, i32, vp]
+    lib.fd_stream_frame_index.argtypes = [vp, i32, ctypes.POINTER(i64)]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
             getattr(lib, name).restype = i32
@@ -144,6 +147,7 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False,
     c.n_refine = int(getattr(cfg, "n_refine", 0)) if c.head_mode else 0
     c.mlp_fp8 = int(getattr(cfg, "mlp_fp8", 0))
     c.record_mlp_amax = int(record_mlp_amax)
+    c.batch = int(getattr(cfg, "batch", 1))
     return c
 
 
@@ -238,8 +242,15 @@ class FlashDecoder:
     def reset(self, stream=None):
         _check(self._lib.fd_reset(self.h, _stream_handle(stream)), "fd_reset")
 
+    def reset_stream(self, b: int, stream=None):
+        """Start a new video in stream b only."""
+        _check(self._lib.fd_reset_stream(self.h, int(b), _stream_handle(stream)),
+               "fd_reset_stream")
+
     def decode_frame(self, latent, out, stream=None):
-        """latent, out: CUDA tensors (or raw device pointers as int)."""
+        """latent [B][C'][H'][W'], out [B][C][r_t][H][W] (B = cfg.batch; the
+        leading axis may be omitted for B = 1): CUDA tensors or raw device
+        pointers as int."""
         lp = latent.data_ptr() if hasattr(latent, "data_ptr") else int(latent)
         op = out.data_ptr() if hasattr(out, "data_ptr") else int(out)
         _check(self._lib.fd_decode_frame(self.h, ctypes.c_void_p(lp), ctypes.c_void_p(op),
@@ -255,9 +266,10 @@ class FlashDecoder:
     def status(self) -> int:
         return int(self._lib.fd_status(self.h))
 
-    def frame_index(self) -> int:
+    def frame_index(self, b: int = 0) -> int:
         t = ctypes.c_int64()
-        _check(self._lib.fd_frame_index(self.h, ctypes.byref(t)), "fd_frame_index")
+        _check(self._lib.fd_stream_frame_index(self.h, int(b), ctypes.byref(t)),
+               "fd_stream_frame_index")
         return t.value
 
     def device_bytes(self) -> int:

@@ -115,6 +115,10 @@ def test_create_rejects_bad_configs_before_touching_the_device():
         setattr(c, field, value)
         s, _ = _create(c)
         assert s == code, (field, value, s, lib.fd_last_error())
+    for value in (0, 65):
+        c = fdb.make_config(base)
+        c.batch = value
+        assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     c = fdb.make_config(bf.replace(mlp_fp8=1), record_mlp_amax=True)
     assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     # FP8 without scale pointers: rejected before any device work
@@ -140,6 +144,8 @@ def test_bad_handle_calls():
     n = ctypes.c_int32()
     assert lib.fd_mlp_fp8_scales(None, None, 0, ctypes.byref(n)) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_debug_block_mlp(None, 0, None, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_reset_stream(None, 0, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_stream_frame_index(None, 0, ctypes.byref(t)) == fdb.FD_ERR_BAD_HANDLE
     # a pointer to memory that is not a handle (magic check)
     junk = (ctypes.c_uint32 * 64)()
     assert lib.fd_reset(ctypes.cast(junk, ctypes.c_void_p), None) == fdb.FD_ERR_BAD_HANDLE
