@@ -381,7 +381,7 @@ fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   const int tiles = ((M + 127) / 128) * (N / BN);
   k->func = f;
   k->grid = dim3(std::min(tiles, num_sms));
-  k->block = dim3(kGemmThreads);
+  k->block = dim3(gemm_threads(KIND));
   k->smem = S::kAlloc;
   return FD_OK;
 }

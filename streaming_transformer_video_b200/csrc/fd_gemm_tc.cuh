@@ -10,9 +10,12 @@
 //               mbarrier (expect_tx) per stage
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=BN,
 //               32 bytes of K per instruction, 4 per stage) and commits
-//   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, one
-//               token row per thread, fused epilogue (fd_epilogue.cuh)
-//               (eight epilogue warps, two per row group, measured no faster)
+//   warps 2..   epilogue: tcgen05.ld of the 128 x BN fp32 accumulator, one
+//               token row per thread, fused epilogue (fd_epilogue.cuh). The
+//               GELU epilogues are arithmetic-bound and get 8 warps (two per
+//               TMEM lane quarter, alternate 64-column chunks; measured 10%
+//               faster); the others wait on memory and keep 4 (8 measured no
+//               faster, and the QKV epilogue would spill)
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the
 // epilogue of tile i overlaps the main loop of tile i+1. Tiles are handed out
 // round-robin over a grid of at most one CTA per SM. Rows past M are read as
@@ -35,14 +38,17 @@ struct TcGemmSmem {
   static constexpr int kAlloc = kBytes + 1024;        // slack for 1024-B alignment
 };
 
-constexpr int kEpiThreads = 128;                       // 4 epilogue warps
-constexpr int kGemmThreads = 64 + kEpiThreads;
+__host__ __device__ constexpr int gemm_epi_threads(int kind) {
+  return (kind == EPI_GELU || kind == EPI_GELU_Q) ? 256 : 128;
+}
+__host__ __device__ constexpr int gemm_threads(int kind) { return 64 + gemm_epi_threads(kind); }
 
 template <int BN, int STAGES, int KIND, int DH, bool F8 = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(KIND), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int K, EpiParams ep, int* status) {
   using S = TcGemmSmem<BN, STAGES>;
+  constexpr int kEpiThreads = gemm_epi_threads(KIND);
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   constexpr uint32_t kTmemCols = 2 * BN;              // power of two: 128, 256 or 512
   static_assert((kTmemCols & (kTmemCols - 1)) == 0, "TMEM columns must be a power of 2");
