@@ -386,11 +386,33 @@ fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   return FD_OK;
 }
 
+// Tile width (BN) of a GEMM: the widest of 256 / 128 / 64 that divides N,
+// except for the residual epilogues (O-projection, MLP-down). These are
+// bound by their epilogue's memory latency. They switch to 128 when 256-wide
+// tiles would occupy fewer CTAs than there are SMs and 128-wide tiles either
+// still fit in one wave, or have a short K (<= 2048) and overflow the wave by
+// at most 1/8. Measured faster for those shapes (480p: O-proj and MLP-down;
+// FlashDecoder-XL 480p: O-proj), not faster for the others (720p O-proj at
+// 1.57 waves, XL MLP-down with K = 6144, every 1080p GEMM). The weight tensor
+// maps use the same rule for their box height.
+int gemm_bn(int kind, int M, int N, int K, int num_sms) {
+  if (N % 256 == 0) {
+    const bool resid = kind == EPI_RESID || kind == EPI_RESID_Q;
+    const long m_tiles = (M + 127) / 128;
+    const long t256 = m_tiles * (N / 256), t128 = m_tiles * (N / 128);
+    if (resid && t256 < num_sms &&
+        (t128 <= num_sms || (K <= 2048 && t128 <= num_sms + num_sms / 8)))
+      return 128;
+    return 256;
+  }
+  return N % 128 == 0 ? 128 : 64;
+}
+
 template <int KIND, bool F8 = false>
-fd_status_t tc_gemm_pick(int M, int N, int num_sms, int* bn, KernelLaunch* k) {
-  if (N % 256 == 0) { *bn = 256; return tc_gemm_launch<256, KIND, F8>(M, N, num_sms, k); }
-  if (N % 128 == 0) { *bn = 128; return tc_gemm_launch<128, KIND, F8>(M, N, num_sms, k); }
-  *bn = 64;
+fd_status_t tc_gemm_pick(int M, int N, int K, int num_sms, int* bn, KernelLaunch* k) {
+  *bn = gemm_bn(KIND, M, N, K, num_sms);
+  if (*bn == 256) return tc_gemm_launch<256, KIND, F8>(M, N, num_sms, k);
+  if (*bn == 128) return tc_gemm_launch<128, KIND, F8>(M, N, num_sms, k);
   return tc_gemm_launch<64, KIND, F8>(M, N, num_sms, k);
 }
 
@@ -459,15 +481,15 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
   if (bf) {
     int bn = 0;
     if (f8) {                     // FP8 MLP: the two MLP GEMMs
-      if (kind == EPI_GELU_Q) FD_TRY((tc_gemm_pick<EPI_GELU_Q, true>(M, N, num_sms, &bn, &k)));
-      else FD_TRY((tc_gemm_pick<EPI_RESID, true>(M, N, num_sms, &bn, &k)));
+      if (kind == EPI_GELU_Q) FD_TRY((tc_gemm_pick<EPI_GELU_Q, true>(M, N, K, num_sms, &bn, &k)));
+      else FD_TRY((tc_gemm_pick<EPI_RESID, true>(M, N, K, num_sms, &bn, &k)));
     } else switch (kind) {
-      case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(M, N, num_sms, &bn, &k)); break;
-      case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(M, N, num_sms, &bn, &k)); break;
-      case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(M, N, num_sms, &bn, &k)); break;
-      case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(M, N, num_sms, &bn, &k)); break;
-      case EPI_RESID_Q: FD_TRY(tc_gemm_pick<EPI_RESID_Q>(M, N, num_sms, &bn, &k)); break;
-      default: FD_TRY(tc_gemm_pick<EPI_FINAL>(M, N, num_sms, &bn, &k)); break;
+      case EPI_QKV: FD_TRY(tc_gemm_pick<EPI_QKV>(M, N, K, num_sms, &bn, &k)); break;
+      case EPI_RESID: FD_TRY(tc_gemm_pick<EPI_RESID>(M, N, K, num_sms, &bn, &k)); break;
+      case EPI_GELU: FD_TRY(tc_gemm_pick<EPI_GELU>(M, N, K, num_sms, &bn, &k)); break;
+      case EPI_UP: FD_TRY(tc_gemm_pick<EPI_UP>(M, N, K, num_sms, &bn, &k)); break;
+      case EPI_RESID_Q: FD_TRY(tc_gemm_pick<EPI_RESID_Q>(M, N, K, num_sms, &bn, &k)); break;
+      default: FD_TRY(tc_gemm_pick<EPI_FINAL>(M, N, K, num_sms, &bn, &k)); break;
     }
     CUtensorMap a = tmA, b = tmB;
     int kk = K;
@@ -932,17 +954,22 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(make_tmap_2d(&h->tm_xb, h->xb, L, D, 128));
     FD_TRY(make_tmap_2d(&h->tm_o, h->o, L, size_t(H) * Dh, 128));
     FD_TRY(make_tmap_2d(&h->tm_h, h->hb, L, h->dff, 128));
-    auto bn_of = [](int N) { return N % 256 == 0 ? 256u : (N % 128 == 0 ? 128u : 64u); };
+    auto bn_of = [&](int N, int kind = EPI_QKV, int K = 0) {
+      return uint32_t(gemm_bn(kind, h->M, N, K, h->num_sms));
+    };
     for (int l = 0; l < NB + NR; ++l) {
       CUtensorMap m;
       FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(h->qkv))); h->tm_wqkv.push_back(m);
-      FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D))); h->tm_wo.push_back(m);
+      FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D, EPI_RESID, H * Dh)));
+      h->tm_wo.push_back(m);
       if (h->fp8) {
         FD_TRY(make_tmap_2d_e4m3(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
-        FD_TRY(make_tmap_2d_e4m3(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+        FD_TRY(make_tmap_2d_e4m3(&m, h->w2[l], D, h->dff, bn_of(D, EPI_RESID, h->dff)));
+        h->tm_w2.push_back(m);
       } else {
         FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
-        FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D))); h->tm_w2.push_back(m);
+        FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D, EPI_RESID, h->dff)));
+        h->tm_w2.push_back(m);
       }
     }
     if (h->fp8) {
