@@ -109,6 +109,25 @@ __device__ __forceinline__ void store_e4m3_64(uint8_t* dst, const float* v, floa
   }
 }
 
+// Four consecutive biases with one 16-byte load (every bias slice an
+// epilogue reads starts on a 32-column boundary of a 256-byte aligned array).
+__device__ __forceinline__ float4 bias4(const float* b, int col) {
+  return __ldg(reinterpret_cast<const float4*>(b + col));
+}
+
+// v[c] = v[c] * s + b[col + c], c < n (n a multiple of 4)
+template <int n>
+__device__ __forceinline__ void scale_bias(float* v, float s, const float* b, int col) {
+#pragma unroll
+  for (int c = 0; c < n; c += 4) {
+    const float4 bb = bias4(b, col + c);
+    v[c] = v[c] * s + bb.x;
+    v[c + 1] = v[c + 1] * s + bb.y;
+    v[c + 2] = v[c + 2] * s + bb.z;
+    v[c + 3] = v[c + 3] * s + bb.w;
+  }
+}
+
 __device__ __forceinline__ void record_amax(unsigned* amax, const float* v) {
   float m = 0.f;
 #pragma unroll
@@ -219,8 +238,7 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
       float* v = acc + hh * DH;
       const int col = col0 + hh * DH;
       const int head = col / DH;
-#pragma unroll
-      for (int d = 0; d < DH; ++d) v[d] = v[d] * rs + __ldg(p.bias + col + d);
+      scale_bias<DH>(v, rs, p.bias, col);
       if (head < p.H) {                                   // query head
         rope_head<DH>(v, n, fs, p);
         T* dst = static_cast<T*>(p.q) + (size_t(head) * p.M + row) * DH;
@@ -247,10 +265,11 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
 #pragma unroll
     for (int c = 0; c < 64; c += 4) {
       float4 o = *reinterpret_cast<const float4*>(x + c);
-      o.x += acc[c + 0] * sc + __ldg(p.bias + col0 + c + 0);
-      o.y += acc[c + 1] * sc + __ldg(p.bias + col0 + c + 1);
-      o.z += acc[c + 2] * sc + __ldg(p.bias + col0 + c + 2);
-      o.w += acc[c + 3] * sc + __ldg(p.bias + col0 + c + 3);
+      const float4 bb = bias4(p.bias, col0 + c);
+      o.x += acc[c + 0] * sc + bb.x;
+      o.y += acc[c + 1] * sc + bb.y;
+      o.z += acc[c + 2] * sc + bb.z;
+      o.w += acc[c + 3] * sc + bb.w;
       *reinterpret_cast<float4*>(x + c) = o;
       acc[c + 0] = o.x; acc[c + 1] = o.y; acc[c + 2] = o.z; acc[c + 3] = o.w;
     }
@@ -268,20 +287,21 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
       p.ssq_out[size_t(row) * parts + col0 / 32 + h] = s;
     }
   } else if constexpr (KIND == EPI_GELU) {
+    scale_bias<64>(acc, rs, p.bias, col0);
 #pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * rs + __ldg(p.bias + col0 + c));
+    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c]);
     store_vec<T, 64>(static_cast<T*>(p.hout) + size_t(row) * p.N + col0, acc);
     if (p.amax) record_amax(p.amax, acc);
   } else if constexpr (KIND == EPI_GELU_Q) {
     const float sc = rs * p.acc_scale;
+    scale_bias<64>(acc, sc, p.bias, col0);
 #pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c] * sc + __ldg(p.bias + col0 + c));
+    for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c]);
     store_e4m3_64(static_cast<uint8_t*>(p.hout) + size_t(row) * p.N + col0, acc, p.q_inv);
   } else if constexpr (KIND == EPI_UP) {
     const int tau = col0 / p.D, c0 = col0 - tau * p.D;
     const size_t r = size_t(tau) * p.M + row;             // row of sub-frame tau
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] += __ldg(p.bias + col0 + c);
+    scale_bias<64>(acc, 1.f, p.bias, col0);
     float* x = p.x32 + r * p.D + c0;
 #pragma unroll
     for (int c = 0; c < 64; c += 4)
@@ -296,8 +316,7 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
       p.ssq_out[r * parts + c0 / 32 + h] = s;
     }
   } else {  // EPI_FINAL
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = acc[c] * rs + __ldg(p.bias + col0 + c);
+    scale_bias<64>(acc, rs, p.bias, col0);
     if (p.P == 16) pixel_scatter<16>(p, row, col0, acc);
     else pixel_scatter<8>(p, row, col0, acc);
   }
