@@ -40,8 +40,8 @@ DEFAULT_CONFIG = "1080p_wan22"
 # profiles/block_1080p_ncu_full.md. Keyed by the sha256 of the kernel source:
 # when the kernel changes the figure no longer applies and is reported as null.
 NCU_ATTN_TRAFFIC = {
-    ("1080p_wan22", "65f32d0d2da8edc88c704bccef57939a8b58ef05a90069521b0e26bd61bcac1a"):
-        117140224 + 10029056,
+    ("1080p_wan22", "57eedbc751f7f407cadbe0cf1292d601e65ddbdfa8315696fefbda8e5e8c64da"):
+        117092864 + 9040128,
 }
 
 

@@ -560,8 +560,8 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.status = status;
     // one 128-query tile per CTA, two CTAs per SM (measured faster than two
     // query tiles sharing one CTA, and than three CTAs with single-buffered S)
-    using A = TcAttnSmem<1>;
-    const void* f = reinterpret_cast<const void*>(&tc_attn_kernel<1>);
+    using A = TcAttnSmem;
+    const void* f = reinterpret_cast<const void*>(&tc_attn_kernel);
     FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
     KernelLaunch k{f, dim3((L + 127) / 128, H, B), dim3(A::kThreads), size_t(A::kAlloc), FD_K_ATTN};
     CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;

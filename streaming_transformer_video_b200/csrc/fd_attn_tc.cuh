@@ -6,26 +6,26 @@
 // are always the contiguous range [0, n_valid*L) and softmax, being
 // invariant to the order of keys, needs no slot bookkeeping.
 //
-// One CTA = one head x QT query tiles of 128 (QT = 1 or 2) of one video
-// stream (blockIdx.z; each stream has its own frame state and cache slab).
-// Keys are consumed in tiles of 64; every K/V stage is shared by the QT
-// query tiles.
-// Warps:
-//   0            TMA: the Q tiles once, then per stage K (64 keys x 64) and
-//                the transposed V (64 dims x 64 keys)
-//   1            TMEM allocator; lane 0 issues, per key tile j,
-//                S_t(j) = Q_t K_j^T (SS form) for every query tile t, then
-//                O_t += P_t(j-1) V_{j-1} (TS form: P read from TMEM)
-//   2 .. 1+4*QT  softmax, one warpgroup per query tile, one query row per
-//                thread: S row from TMEM, base-2 online softmax with lazy
-//                rescaling (O is rescaled in TMEM only when the running max
-//                grows by more than 2^8), P packed to bf16 into TMEM
-// S and P are double-buffered per query tile, so the softmax of tile j runs
-// while the tensor core still computes S(j+1) and O += P(j-1) V(j-1); the
-// only waits on the critical path are for data two tiles old.
-// TMEM columns (64 fp32 S columns, 32 packed-bf16 P columns per buffer):
-//   S[t][b] at 64 (2t + b), O_t at 64 (2 QT + t), P[t][b] at 64 (3 QT) + 32 (2t + b).
-// Keys past n_valid*L inside the last tile get probability 0.
+// One CTA = one head x 128 queries of one video stream (blockIdx.z; each
+// stream has its own frame state and cache slab); 192 threads, 2 CTAs per SM.
+// Keys are consumed in tiles of 64.
+//   warp 0      TMA: Q once, then per stage K (64 keys x 64) and the
+//               transposed V (64 dims x 64 keys)
+//   warp 1      TMEM allocator; lane 0 issues S(j) = Q K_j^T (SS form) into
+//               S buffer j mod 3 once O += P(j-3) V(j-3) has read that
+//               buffer; lane 1 issues O += P(j) V_j (TS form: P read from
+//               TMEM) as soon as P(j) is written, then releases the K/V stage.
+//               Each lane's tcgen05.commit tracks only its own MMAs.
+//   warps 2..5  softmax, one query row per thread: S row from TMEM, base-2
+//               online softmax with lazy rescaling (O is rescaled in TMEM only
+//               when the running max grows by more than 2^8), P packed to bf16
+//               and written over the S it came from
+// TMEM columns: S buffer b (b < 3) at 64 b, with P(j) in the first 32 columns
+// of its buffer; O at 192. S runs up to three tiles ahead of the softmax,
+// whose only synchronisation per tile is the wait for S(j) and the arrival
+// that hands P(j) to the PV issuer. (Measured against two S buffers with
+// separate P columns: bit-identical output, equal time at 1080p, 7% faster
+// at 480p.) Keys past n_valid*L inside the last tile get probability 0.
 #pragma once
 
 #include "fd_ptx.cuh"
@@ -41,23 +41,6 @@ struct TcAttnParams {
   float scale_log2;   // log2(e) / sqrt(64)
   const FrameState* fs;
   int* status;
-};
-
-template <int QT>
-struct TcAttnSmem {
-  static constexpr int kStages = QT == 2 ? 8 : 4;
-  static constexpr int kQ = 0;                                // QT x 16 KB
-  static constexpr int kKV = QT * 16384;                      // stages x (K 8 KB + V^T 8 KB)
-  static constexpr int kKVStage = 16384;
-  static constexpr int kBar = kKV + kStages * kKVStage;
-  // q_full, kv_full[ST], kv_empty[ST], then per tile: s_full[2], s_free[2],
-  // p_full[2], p_free[2], o_final
-  static constexpr int kNumBars = 1 + 2 * kStages + 9 * QT;
-  static constexpr int kBytes = kBar + kNumBars * 8 + 16;
-  static constexpr int kAlloc = kBytes + 1024;
-  static constexpr int kThreads = 64 + 128 * QT;
-  static constexpr int kTmemCols = QT == 2 ? 512 : 256;
-  static constexpr int kMinBlocks = QT == 2 ? 1 : 2;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -125,34 +108,44 @@ __device__ __forceinline__ float exp_pack64(const float* x, float sc, float m, u
   return a0.x + a0.y;
 }
 
-template <int QT>
-__global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMinBlocks)
+struct TcAttnSmem {
+  static constexpr int kStages = 4;
+  static constexpr int kQ = 0;                                // 16 KB
+  static constexpr int kKV = 16384;                           // stages x (K 8 KB + V^T 8 KB)
+  static constexpr int kKVStage = 16384;
+  static constexpr int kBar = kKV + kStages * kKVStage;
+  // q_full, kv_full[ST], kv_empty[ST], s_full[3], p_full[3], p_free[3], o_final
+  static constexpr int kNumBars = 1 + 2 * kStages + 10;
+  static constexpr int kBytes = kBar + kNumBars * 8 + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kThreads = 192;
+  static constexpr int kTmemCols = 256;
+};
+
+__global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
     tc_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, TcAttnParams p) {
-  using S = TcAttnSmem<QT>;
+  using S = TcAttnSmem;
   constexpr int ST = S::kStages;
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64);   // 128 queries x 64 keys
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, 64);   // 128 queries x 64 dims
-  constexpr uint32_t kColO = 64 * 2 * QT, kColP = 64 * 3 * QT;
+  constexpr uint32_t kColO = 192;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* kv_full = q_full + 1;
   uint64_t* kv_empty = kv_full + ST;
-  uint64_t* tb = kv_empty + ST;                 // per tile t: 9 barriers at tb + 9 t
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tb + 9 * QT);
+  uint64_t* s_full = kv_empty + ST;                 // [3]
+  uint64_t* p_full = s_full + 3;                    // [3]
+  uint64_t* p_free = p_full + 3;                    // [3]
+  uint64_t* o_final = p_free + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto s_full = [&](int t, int b) { return tb + 9 * t + b; };
-  auto s_free = [&](int t, int b) { return tb + 9 * t + 2 + b; };
-  auto p_full = [&](int t, int b) { return tb + 9 * t + 4 + b; };
-  auto p_free = [&](int t, int b) { return tb + 9 * t + 6 + b; };
-  auto o_final = [&](int t) { return tb + 9 * t + 8; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (128 * QT), h = blockIdx.y, bs = blockIdx.z;
+  const int q0 = blockIdx.x * 128, h = blockIdx.y, bs = blockIdx.z;
   const int g = h / (p.H / p.G);
   const int lg = (p.layer * p.B + bs) * p.G + g;
   const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
@@ -161,13 +154,10 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < ST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int t = 0; t < QT; ++t) {
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(s_full(t, b), 1); mbar_init(s_free(t, b), 128);
-        mbar_init(p_full(t, b), 128); mbar_init(p_free(t, b), 1);
-      }
-      mbar_init(o_final(t), 1);
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 128); mbar_init(&p_free[b], 1);
     }
+    mbar_init(o_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmQ); prefetch_tensormap(&tmK); prefetch_tensormap(&tmV);
@@ -180,9 +170,8 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
 
   if (warp == 0) {
     if (lane == 0) {                                       // ---- TMA producer
-      mbar_arrive_expect_tx(q_full, QT * 16384);
-      for (int t = 0; t < QT; ++t)
-        tma_load_4d(smem + S::kQ + t * 16384, &tmQ, 0, q0 + t * 128, bs, h, q_full);
+      mbar_arrive_expect_tx(q_full, 16384);
+      tma_load_4d(smem + S::kQ, &tmQ, 0, q0, bs, h, q_full);
       for (int j = 0; j < n_kt; ++j) {
         const int st = j % ST;
         if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
@@ -193,79 +182,65 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
       }
     }
   } else if (warp == 1) {
-    // Two MMA issuers, so S(j+1) never waits behind O += P(j-1) V(j-1):
-    // lane 0 issues S_t(j) = Q_t K_j^T as soon as an S buffer is free;
-    // lane 1 issues O_t += P_t(j) V_j as soon as P_t(j) is written, then
-    // releases the K/V stage (S(j) precedes P(j), so K is no longer read).
-    // Each lane's tcgen05.commit tracks only its own MMAs.
     if (lane == 0) {                                       // ---- S issuer
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < n_kt; ++j) {
-        const int st = j % ST, b = j & 1;
+        const int st = j % ST, b = j % 3;
         if (!mbar_wait(&kv_full[st], (j / ST) & 1, abort_flag, p.status)) break;
+        // buffer b last held P(j-3): O += P(j-3) V(j-3) must have read it
+        if (j >= 3 && !mbar_wait(&p_free[b], ((j / 3) - 1) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t sq = smem_u32(smem + S::kQ);
         const uint32_t sk = smem_u32(smem + S::kKV + st * S::kKVStage);
-        for (int t = 0; t < QT; ++t) {
-          if (!mbar_wait(s_free(t, b), ((j >> 1) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sq = smem_u32(smem + S::kQ + t * 16384);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ss(tmem_base + 64 * (2 * t + b), sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k,
-                      kIdescS, k != 0);
-          tc_commit(s_full(t, b));
-        }
+        for (int k = 0; k < 4; ++k)
+          tc_mma_ss(tmem_base + 64 * b, sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k, kIdescS,
+                    k != 0);
+        tc_commit(&s_full[b]);
       }
     } else if (lane == 1) {                                // ---- PV issuer
       bool ok = true;
       for (int i = 0; ok && i < n_kt; ++i) {
-        const int b = i & 1;
+        const int b = i % 3;
+        if (!mbar_wait(&p_full[b], (i / 3) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
         const uint32_t sv = smem_u32(smem + S::kKV + (i % ST) * S::kKVStage + 8192);
-        for (int t = 0; t < QT; ++t) {
-          if (!mbar_wait(p_full(t, b), (i >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_tm = tmem_base + kColP + 32 * (2 * t + b);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem_base + kColO + 64 * t, a_tm + 8 * k, sw128_desc(sv) + 2 * k, kIdescO,
-                      (i | k) != 0);
-          tc_commit(p_free(t, b));
-        }
-        if (ok) tc_commit(&kv_empty[i % ST]);
+        for (int k = 0; k < 4; ++k)
+          tc_mma_ts(tmem_base + kColO, tmem_base + 64 * b + 8 * k, sw128_desc(sv) + 2 * k, kIdescO,
+                    (i | k) != 0);
+        tc_commit(&p_free[b]);
+        tc_commit(&kv_empty[i % ST]);
       }
-      if (ok)
-        for (int t = 0; t < QT; ++t) tc_commit(o_final(t));
+      if (ok) tc_commit(o_final);
     }
-  } else {                                                 // ---- softmax warpgroups
-    const int t = (warp - 2) >> 2;                         // query tile of this warpgroup
+  } else {                                                 // ---- softmax warps
     const int quarter = warp & 3;                          // TMEM lanes 32*quarter ..
     const int r = quarter * 32 + lane;                     // query row within the tile
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t tm_o = tmem_base + lane_off + kColO + 64 * t;
+    const uint32_t tm_o = tmem_base + lane_off + kColO;
     const float sc = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait_warp(s_full(t, b), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      const int b = j % 3;
+      if (!mbar_wait_warp(&s_full[b], (j / 3) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
       float x[64];
       {
         uint32_t r0[32], r1[32];
-        const uint32_t tm_s = tmem_base + lane_off + 64 * (2 * t + b);
+        const uint32_t tm_s = tmem_base + lane_off + 64 * b;
         tmem_ld32(tm_s, r0); tmem_ld32(tm_s + 32, r1);
         tmem_ld_wait();
         reg_fence(r0); reg_fence(r1);
 #pragma unroll
         for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
       }
-      tc_fence_before();
-      mbar_arrive(s_free(t, b));
       const int valid = n_keys - j * 64;                   // keys of this tile in range
       if (valid < 64) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
       }
-      // row max of the raw scores (the scale is positive)
       float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
 #pragma unroll
       for (int c = 6; c < 62; c += 4) { m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]); }
@@ -278,14 +253,10 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
       if (rescale) { m_ref = mx; l *= corr; }
       uint32_t pk[32];
       l += exp_pack64(x, sc, m_ref, pk);
-      // P buffer b was last read by the MMA of tile j-2
-      if (j >= 2) {
-        if (!mbar_wait_warp(p_free(t, b), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-      }
       if (__any_sync(0xffffffffu, rescale)) {
-        // O_t *= corr (rare): every earlier O += P V must have landed first
-        if (!mbar_wait_warp(p_free(t, b ^ 1), ((j - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        // O *= corr (rare): every earlier O += P V must have landed first
+        const int jp = j - 1;
+        if (!mbar_wait_warp(&p_free[jp % 3], (jp / 3) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t o0[32], o1[32];
         tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
@@ -298,18 +269,18 @@ __global__ void __launch_bounds__(TcAttnSmem<QT>::kThreads, TcAttnSmem<QT>::kMin
         }
         tmem_st32(tm_o, o0); tmem_st32(tm_o + 32, o1);
       }
-      tmem_st32(tmem_base + lane_off + kColP + 32 * (2 * t + b), pk);
+      tmem_st32(tmem_base + lane_off + 64 * b, pk);        // P over the S it came from
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full(t, b));
+      mbar_arrive(&p_full[b]);
     }
-    if (ok && mbar_wait_warp(o_final(t), 0, abort_flag, p.status)) {
+    if (ok && mbar_wait_warp(o_final, 0, abort_flag, p.status)) {
       tc_fence_after();
       uint32_t o0[32], o1[32];
       tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
       tmem_ld_wait();
       reg_fence(o0); reg_fence(o1);
-      const int row = q0 + t * 128 + r;
+      const int row = q0 + r;
       if (row < p.L) {
         const float inv = 1.f / l;
         float v[64];
