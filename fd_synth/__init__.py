@@ -65,6 +65,8 @@ class FDConfig:
     mlp_fp8: int = 0
     # video streams decoded together per step (each its own video and cache)
     batch: int = 1
+    # bf16 attention key splitting: 0 = automatic, 1..4 forced
+    attn_splits: int = 0
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property

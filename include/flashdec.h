@@ -105,6 +105,11 @@ typedef struct {
                             call takes one latent frame of each stream; each
                             stream has its own frame counter and ring slots
                             ([FD] Eq. 1 carries a batch dimension B)          */
+  int32_t attn_splits;   /* bf16 attention: split every (query tile, head)'s key
+                            range over this many CTAs and combine the partial
+                            results (1 .. 4); 0 = chosen from the launch's fit
+                            to the GPU's CTA slots. Results differ from 1 only
+                            by floating-point summation order.               */
 } fd_config;
 
 /*

@@ -195,6 +195,9 @@ struct fd_handle {
   int fp8 = 0;                      // 1: FP8 E4M3 MLP GEMMs
   int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
   int B = 1, M = 0;                 // video streams; GEMM rows M = B L
+  int n_split = 1;                  // attention key splitting (1: off)
+  float *part_o = nullptr, *part_ml = nullptr;   // its partial results
+  int* split_ctr = nullptr;
   int fs_stride = 1;                // FrameStates per stream: 1 (+ r_t, paper head)
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
   int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
@@ -555,6 +558,10 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.B = B;
     ap.fs_stride = fs_stride;
     ap.layer = io.layer;
+    ap.n_split = n_split;
+    ap.part_o = part_o;
+    ap.part_ml = part_ml;
+    ap.counter = split_ctr;
     ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
     ap.fs = io.fs;
     ap.status = status;
@@ -563,7 +570,8 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     using A = TcAttnSmem;
     const void* f = reinterpret_cast<const void*>(&tc_attn_kernel);
     FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
-    KernelLaunch k{f, dim3((L + 127) / 128, H, B), dim3(A::kThreads), size_t(A::kAlloc), FD_K_ATTN};
+    KernelLaunch k{f, dim3((L + 127) / 128, H, B * n_split), dim3(A::kThreads), size_t(A::kAlloc),
+                   FD_K_ATTN};
     CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;
     void* args[] = {&a, &b, &c, &ap};
     FD_TRY(add_kernel(k, args));
@@ -782,6 +790,8 @@ fd_status_t validate(const fd_config* c) {
   if (L * (c->window + 1) > (1LL << 30))
     return fail(FD_ERR_UNSUPPORTED, "config: window of %lld tokens is too large",
                 L * (c->window + 1));
+  if (c->attn_splits < 0 || c->attn_splits > 4)
+    return fail(FD_ERR_INVALID_ARG, "config: attn_splits must be 0 .. 4 (got %d)", c->attn_splits);
   if (c->batch < 1 || c->batch > fd::kMaxStreams)
     return fail(FD_ERR_INVALID_ARG, "config: batch must be 1 .. %d (got %d)", fd::kMaxStreams, c->batch);
   if (c->kernel_timing < 0 || c->kernel_timing > 2)
@@ -922,6 +932,27 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   if (c.record_mlp_amax) {
     h->n_amax = 2 * (NB + NR);
     FD_TRY(h->alloc(&h->amax, size_t(h->n_amax) * 4));
+  }
+  // attention key splitting: chosen by the attention launch's fit to the CTA
+  // slots (2 per SM): est(s) = waves(s units) / s, plus 4% per extra split for
+  // the partial writes and the combine
+  if (h->bf) {
+    const long units = long((h->L + 127) / 128) * H * h->B;
+    const long slots = 2L * h->num_sms;
+    h->n_split = c.attn_splits;
+    if (h->n_split == 0) {
+      double best = 1e30;
+      for (int sp = 1; sp <= 3; ++sp) {
+        const double est = double((units * sp + slots - 1) / slots) / sp * (1.0 + 0.04 * (sp - 1));
+        if (est < best - 1e-9) { best = est; h->n_split = sp; }
+      }
+    }
+    if (h->n_split > 1) {
+      FD_TRY(h->alloc(&h->part_o, size_t(units) * h->n_split * 128 * 64 * 4));
+      FD_TRY(h->alloc(&h->part_ml, size_t(units) * h->n_split * 128 * 2 * 4));
+      FD_TRY(h->alloc(&h->split_ctr, size_t(units) * 4));
+      FD_CUDA(cudaMemset(h->split_ctr, 0, size_t(units) * 4));
+    }
   }
   FD_TRY(h->alloc(&h->ctr, size_t(h->B) * 8));
   FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * h->fs_stride * h->B));

@@ -26,6 +26,14 @@
 // that hands P(j) to the PV issuer. (Measured against two S buffers with
 // separate P columns: bit-identical output, equal time at 1080p, 7% faster
 // at 480p.) Keys past n_valid*L inside the last tile get probability 0.
+//
+// Key splitting (n_split > 1, for launches that fill the GPU's CTA slots
+// poorly): the key tiles of every (query tile, head, stream) are divided into
+// n_split contiguous ranges, one CTA each (blockIdx.z = stream * n_split +
+// split). Each CTA writes its unnormalised O, running max and sum to scratch
+// (part_o, part_ml), fences, and counts itself in counter[unit]; the CTA that
+// arrives last combines the partials in split order (deterministic), writes O
+// and resets the counter for the next launch. No CTA waits for another.
 #pragma once
 
 #include "fd_ptx.cuh"
@@ -41,6 +49,11 @@ struct TcAttnParams {
   float scale_log2;   // log2(e) / sqrt(64)
   const FrameState* fs;
   int* status;
+  // key splitting (n_split 1: off); unit = (stream * H + head) * gridDim.x + query tile
+  int n_split;
+  float* part_o;      // [unit][n_split][128][64] unnormalised O
+  float* part_ml;     // [unit][n_split][128][2] running max (log2 domain), sum
+  int* counter;       // [unit] CTAs of the unit done so far (0 between launches)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -143,13 +156,18 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
   uint64_t* o_final = p_free + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 128, h = blockIdx.y, bs = blockIdx.z;
+  const int q0 = blockIdx.x * 128, h = blockIdx.y;
+  const int bs = blockIdx.z / p.n_split, split = blockIdx.z - bs * p.n_split;
   const int g = h / (p.H / p.G);
   const int lg = (p.layer * p.B + bs) * p.G + g;
   const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
-  const int n_kt = (n_keys + 63) / 64;
+  const int n_kt_all = (n_keys + 63) / 64;
+  // this CTA's key tiles: [j0, j0 + n_kt) (all of them without splitting)
+  const int j0 = split * n_kt_all / p.n_split;
+  const int n_kt = (split + 1) * n_kt_all / p.n_split - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -177,8 +195,8 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
         if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* kv = smem + S::kKV + st * S::kKVStage;
         mbar_arrive_expect_tx(&kv_full[st], S::kKVStage);
-        tma_load_3d(kv, &tmK, 0, j * 64, lg, &kv_full[st]);
-        tma_load_3d(kv + 8192, &tmV, j * 64, 0, lg, &kv_full[st]);
+        tma_load_3d(kv, &tmK, 0, (j0 + j) * 64, lg, &kv_full[st]);
+        tma_load_3d(kv + 8192, &tmV, (j0 + j) * 64, 0, lg, &kv_full[st]);
       }
     }
   } else if (warp == 1) {
@@ -236,7 +254,7 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
 #pragma unroll
         for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(r0[c]); x[32 + c] = __uint_as_float(r1[c]); }
       }
-      const int valid = n_keys - j * 64;                   // keys of this tile in range
+      const int valid = n_keys - (j0 + j) * 64;            // keys of this tile in range
       if (valid < 64) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
@@ -274,23 +292,78 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
-    if (ok && mbar_wait_warp(o_final, 0, abort_flag, p.status)) {
+    // the o_final commit is awaited even for an empty key range, so that no
+    // asynchronous arrival can land after the CTA has exited
+    const bool have_o = ok && mbar_wait_warp(o_final, 0, abort_flag, p.status);
+    float v[64];
+    if (have_o && n_kt > 0) {
       tc_fence_after();
       uint32_t o0[32], o1[32];
       tmem_ld32(tm_o, o0); tmem_ld32(tm_o + 32, o1);
       tmem_ld_wait();
       reg_fence(o0); reg_fence(o1);
-      const int row = q0 + r;
-      if (row < p.L) {
-        const float inv = 1.f / l;
-        float v[64];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          v[c] = __uint_as_float(o0[c]) * inv;
-          v[32 + c] = __uint_as_float(o1[c]) * inv;
-        }
+      for (int c = 0; c < 32; ++c) { v[c] = __uint_as_float(o0[c]); v[32 + c] = __uint_as_float(o1[c]); }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) v[c] = 0.f;
+      m_ref = -INFINITY;
+      l = 0.f;
+    }
+    const int row = q0 + r;
+    if (p.n_split == 1) {
+      if (have_o && row < p.L) {
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] *= inv;
         store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
                                 size_t(h) * 64, v);
+      }
+    } else {
+      // this key range's partial result
+      const size_t unit = (size_t(bs) * p.H + h) * gridDim.x + blockIdx.x;
+      const size_t prow = (unit * p.n_split + split) * 128 + r;
+      float4* po = reinterpret_cast<float4*>(p.part_o + prow * 64);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) po[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(m_ref, l);
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");      // the four softmax warps
+      if (threadIdx.x == 64) {
+        const int done = atomicAdd(p.counter + unit, 1);
+        const int last = done == p.n_split - 1;
+        if (last) p.counter[unit] = 0;                    // ready for the next launch
+        *last_flag = last;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*last_flag) {
+        __threadfence();
+        // combine the n_split partials of this row in split order
+        float mstar = -INFINITY;
+        for (int sp = 0; sp < p.n_split; ++sp)
+          mstar = fmaxf(mstar, reinterpret_cast<const float2*>(p.part_ml)[(unit * p.n_split + sp) * 128 + r].x);
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] = 0.f;
+        for (int sp = 0; sp < p.n_split; ++sp) {
+          const size_t q = (unit * p.n_split + sp) * 128 + r;
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + q);
+          const float w = ex2(ml.x - mstar);              // 0 for an empty range
+          lsum += w * ml.y;
+          const float4* pq = reinterpret_cast<const float4*>(p.part_o + q * 64);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float4 t = __ldcg(pq + c);
+            v[4 * c] += w * t.x; v[4 * c + 1] += w * t.y; v[4 * c + 2] += w * t.z; v[4 * c + 3] += w * t.w;
+          }
+        }
+        if (row < p.L) {
+          const float inv = 1.f / lsum;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) v[c] *= inv;
+          store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
+                                  size_t(h) * 64, v);
+        }
       }
     }
   }

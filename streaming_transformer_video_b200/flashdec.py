@@ -39,7 +39,8 @@ class FDConfigC(ctypes.Structure):
         ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
         ("kernel_timing", ctypes.c_int32), ("head_mode", ctypes.c_int32),
         ("n_refine", ctypes.c_int32), ("mlp_fp8", ctypes.c_int32),
-        ("record_mlp_amax", ctypes.c_int32), ("batch", ctypes.c_int32)]
+        ("record_mlp_amax", ctypes.c_int32), ("batch", ctypes.c_int32),
+        ("attn_splits", ctypes.c_int32)]
 
 
 _PF = ctypes.POINTER(ctypes.c_float)
@@ -148,6 +149,7 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False,
     c.mlp_fp8 = int(getattr(cfg, "mlp_fp8", 0))
     c.record_mlp_amax = int(record_mlp_amax)
     c.batch = int(getattr(cfg, "batch", 1))
+    c.attn_splits = int(getattr(cfg, "attn_splits", 0))
     return c
 
 

@@ -119,6 +119,10 @@ def test_create_rejects_bad_configs_before_touching_the_device():
         c = fdb.make_config(base)
         c.batch = value
         assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
+    for value in (-1, 5):
+        c = fdb.make_config(base)
+        c.attn_splits = value
+        assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     c = fdb.make_config(bf.replace(mlp_fp8=1), record_mlp_amax=True)
     assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     # FP8 without scale pointers: rejected before any device work

@@ -269,3 +269,33 @@ def test_xl_gqa_480p_full_depth_frames_0_to_2_match_oracle():
     got = gpu_decode(cfg, w, z)
     ref = oracle_decode(cfg, w, z)
     assert_close(cfg, got, ref)
+
+
+# ---------------------------------------------------------------- key splitting
+@pytest.mark.parametrize("kw", [
+    dict(attn_splits=1),
+    dict(attn_splits=2),
+    dict(attn_splits=4, window=3, frames=6),
+    dict(attn_splits=3, grid_h=1, grid_w=1),                  # 1 key tile: empty ranges
+    dict(attn_splits=3, n_heads=8, n_kv_heads=1, d_model=512),
+    dict(attn_splits=2, head="paper", n_refine=2, window=1, frames=3),
+])
+def test_attention_key_splitting_matches_oracle(kw):
+    # each (query tile, head) split over several CTAs, partial results
+    # combined by the last one (flash-decoding style), against the oracle
+    cfg = small_bf16(**kw)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    assert_close(cfg, gpu_decode(cfg, w, z), oracle_decode(cfg, w, z))
+
+
+def test_attention_key_splitting_is_deterministic():
+    cfg = small_bf16(attn_splits=3, frames=4)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    a, dec = gpu_decode(cfg, w, z, keep=True)
+    b = gpu_decode(cfg, w, z, dec=dec)                      # same handle, reset, again
+    dec.close()
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(gpu_decode(cfg, w, z), a)  # a fresh handle
+
