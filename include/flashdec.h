@@ -276,6 +276,31 @@ FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* 
                                    int32_t cap, int32_t* n_out);
 
 /*
+ * fd_decode_frame without the handle's attention scratch (the paper has no
+ * counterpart: this is a deployment variant of this library). Identical
+ * results to fd_decode_frame. When the handle's attention splits its key
+ * ranges (fd_config.attn_splits, or the automatic choice), the partial
+ * results and counters of that split live in one fixed, statically sized
+ * device array of this library (8 MiB) instead of memory allocated by
+ * fd_create; this call allocates nothing. Handles whose split needs more than
+ * 8 MiB ((L/128 rounded up) x heads x batch x splits x 33 KB, plus 4 bytes per
+ * unit) get FD_ERR_UNSUPPORTED; handles that do not split simply run
+ * fd_decode_frame.
+ *  - The array is shared by every handle and stream of the process on that
+ *    device: calls that overlap in time (different streams, threads or
+ *    handles, or an fd_decode_frame_static_scratch still running on the GPU
+ *    when another is enqueued on a different stream) race on it and give wrong
+ *    results. Serialise them on one stream.
+ *  - The first call on each device resolves the array's address
+ *    (cudaGetSymbolAddress); make it outside any CUDA stream capture. Each
+ *    call also updates the attention nodes of the handle's frame graph before
+ *    and after enqueueing it, so it must not be captured either.
+ * Errors as for fd_decode_frame, plus FD_ERR_UNSUPPORTED for oversize.
+ */
+FD_API fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent_frame,
+                                                  void* out_pixels, void* stream);
+
+/*
  * Static FP8 scales from the calibration recorded by a handle created with
  * record_mlp_amax = 1 ([FD] Sec. 4.6: static calibration): for every block
  * (backbone, then refinement), scales_out[2 l] = fp32(max |x| / 448) and

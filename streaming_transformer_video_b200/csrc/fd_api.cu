@@ -22,6 +22,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -173,6 +174,15 @@ struct BlockIO {
   const FrameState* fs;     // stream 0's state of the (sub-)frame; stride fs_stride
 };
 
+// An attention node of the frame graph, kept so that its scratch pointers can
+// be redirected (fd_decode_frame_static_scratch).
+struct AttnNode {
+  cudaGraphNode_t node = nullptr;
+  KernelLaunch launch{};
+  CUtensorMap tmQ{}, tmK{}, tmV{};
+  TcAttnParams p{};
+};
+
 // A kernel node that writes the caller's pixel buffer (patched per call).
 struct OutNode {
   cudaGraphNode_t node = nullptr;
@@ -245,6 +255,7 @@ struct fd_handle {
   KernelLaunch embed_launch{};
   EmbedParams embed_p{};
   std::vector<OutNode> out_nodes;       // kernels writing the pixel buffer
+  std::vector<AttnNode> attn_nodes;     // tcgen05 attention launches
   const void* cur_latent = nullptr;
   void* cur_out = nullptr;
   std::vector<cudaEvent_t> events;
@@ -367,6 +378,7 @@ struct fd_handle {
   fd_status_t add_block(int wi, const BlockIO& io);
   fd_status_t add_post_attention(int wi, const BlockIO& io);
   EpiParams base_epi(const BlockIO& io) const;
+  size_t split_units() const { return size_t((L + 127) / 128) * cfg.n_heads * B; }
   BlockIO backbone_io(int layer);
   BlockIO subframe_io(int tau, int layer);
 };
@@ -574,7 +586,14 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
                    FD_K_ATTN};
     CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;
     void* args[] = {&a, &b, &c, &ap};
-    FD_TRY(add_kernel(k, args));
+    AttnNode an;
+    FD_TRY(add_kernel(k, args, &an.node));
+    an.launch = k;
+    an.tmQ = a;
+    an.tmK = b;
+    an.tmV = c;
+    an.p = ap;
+    attn_nodes.push_back(an);
   } else {
     AttnParams ap{};
     ap.q = q;
@@ -1159,6 +1178,7 @@ fd_status_t fd_reset(fd_handle* h, void* stream) {
   FD_CUDA(cudaMemsetAsync(h->ctr, 0, size_t(h->B) * 8, s));
   FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
   if (h->amax) FD_CUDA(cudaMemsetAsync(h->amax, 0, size_t(h->n_amax) * 4, s));
+  if (h->split_ctr) FD_CUDA(cudaMemsetAsync(h->split_ctr, 0, h->split_units() * 4, s));
   h->last_stream = s;
   return FD_OK;
 }
@@ -1353,6 +1373,72 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
     st = fail(FD_ERR_CUDA, "fd_debug_block_mlp: %s", cudaGetErrorString(e));
   }
   return st;
+}
+
+}  // extern "C"
+
+// Fixed device scratch of fd_decode_frame_static_scratch: the attention
+// key-splitting partials and counters of one frame, for handles whose need fits
+// (modest configurations). Zero at module load; every launch leaves its
+// counters at zero again.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_base[64] = {};                 // per device, from cudaGetSymbolAddress
+}  // namespace
+
+extern "C" {
+
+fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent, void* out,
+                                           void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame_static_scratch: invalid handle");
+  if (h->n_split == 1 || h->attn_nodes.empty())       // this handle's attention uses no scratch
+    return fd_decode_frame(h, latent, out, stream);
+  const size_t units = h->split_units();
+  const size_t o_bytes = units * h->n_split * 128 * 64 * 4;
+  const size_t ml_bytes = units * h->n_split * 128 * 2 * 4;
+  const size_t need = round_up(o_bytes, 256) + round_up(ml_bytes, 256) + units * 4;
+  if (need > kStaticScratchBytes)
+    return fail(FD_ERR_UNSUPPORTED,
+                "fd_decode_frame_static_scratch: attention scratch of %zu bytes exceeds the fixed %zu",
+                need, kStaticScratchBytes);
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FD_ERR_UNSUPPORTED, "fd_decode_frame_static_scratch: device %d", dev);
+  char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_base[dev]) FD_CUDA(cudaGetSymbolAddress(&g_static_base[dev], g_static_scratch));
+    base = static_cast<char*>(g_static_base[dev]);
+  }
+  // point every attention node at the fixed scratch, replay, point them back
+  // (a graph parameter update affects launches made after it only)
+  auto set = [&](bool fixed) -> fd_status_t {
+    for (AttnNode& an : h->attn_nodes) {
+      TcAttnParams ap = an.p;
+      if (fixed) {
+        ap.part_o = reinterpret_cast<float*>(base);
+        ap.part_ml = reinterpret_cast<float*>(base + round_up(o_bytes, 256));
+        ap.counter = reinterpret_cast<int*>(base + round_up(o_bytes, 256) + round_up(ml_bytes, 256));
+      }
+      CUtensorMap a = an.tmQ, b = an.tmK, c = an.tmV;
+      void* args[] = {&a, &b, &c, &ap};
+      cudaKernelNodeParams np{};
+      np.func = const_cast<void*>(an.launch.func);
+      np.gridDim = an.launch.grid;
+      np.blockDim = an.launch.block;
+      np.sharedMemBytes = unsigned(an.launch.smem);
+      np.kernelParams = args;
+      FD_CUDA(cudaGraphExecKernelNodeSetParams(h->exec, an.node, &np));
+    }
+    return FD_OK;
+  };
+  FD_TRY(set(true));
+  const fd_status_t st = fd_decode_frame(h, latent, out, stream);
+  const fd_status_t back = set(false);
+  return st != FD_OK ? st : back;
 }
 
 fd_status_t fd_mlp_fp8_scales(fd_handle* h, float* scales_out, int32_t cap, int32_t* n_out) {

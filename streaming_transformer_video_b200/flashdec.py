@@ -28,7 +28,7 @@ EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
            "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
            "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp",
-           "fd_reset_stream", "fd_stream_frame_index"]
+           "fd_reset_stream", "fd_stream_frame_index", "fd_decode_frame_static_scratch"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -86,6 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_mlp_fp8_scales.argtypes = [vp, _PF, i32, ctypes.POINTER(i32)]
     lib.fd_debug_block_mlp.argtypes = [vp, i32, _PF, _PF]
     lib.fd_reset_stream.argtypes = [vp, i32, vp]
+    lib.fd_decode_frame_static_scratch.argtypes = [vp, vp, vp, vp]
     lib.fd_stream_frame_index.argtypes = [vp, i32, ctypes.POINTER(i64)]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
@@ -257,6 +258,16 @@ class FlashDecoder:
         op = out.data_ptr() if hasattr(out, "data_ptr") else int(out)
         _check(self._lib.fd_decode_frame(self.h, ctypes.c_void_p(lp), ctypes.c_void_p(op),
                                          _stream_handle(stream)), "fd_decode_frame")
+
+    def decode_frame_static_scratch(self, latent, out, stream=None):
+        """decode_frame whose attention scratch is the library's fixed device
+        array (no allocation; calls must not overlap in time)."""
+        lp = latent.data_ptr() if hasattr(latent, "data_ptr") else int(latent)
+        op = out.data_ptr() if hasattr(out, "data_ptr") else int(out)
+        _check(self._lib.fd_decode_frame_static_scratch(self.h, ctypes.c_void_p(lp),
+                                                        ctypes.c_void_p(op),
+                                                        _stream_handle(stream)),
+               "fd_decode_frame_static_scratch")
 
     def decode_frame_host(self, latent, out, stream=None):
         """latent, out: host buffers (pinned tensors or numpy arrays)."""

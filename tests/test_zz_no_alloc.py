@@ -1,0 +1,101 @@
+"""fd_decode_frame_static_scratch: the frame step with the attention's
+key-splitting scratch in the library's fixed device array instead of memory
+allocated by fd_create. It must give exactly what fd_decode_frame gives, on
+consecutive calls, leave the handle's own graph as it was, and refuse handles
+whose scratch does not fit.
+"""
+import numpy as np
+import pytest
+
+import fd_synth
+
+from gpu_util import small_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from streaming_transformer_video_b200 import lib
+    lib()
+
+
+def _frames(cfg, z):
+    import torch
+    lat = torch.from_numpy(z).to(torch.bfloat16).cuda()
+    outs = [torch.empty(cfg.out_shape, dtype=torch.bfloat16, device="cuda") for _ in range(z.shape[0])]
+    return lat, outs
+
+
+def test_static_scratch_equals_decode_frame_on_two_calls_in_a_row():
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder
+    cfg = small_bf16(attn_splits=3, frames=3)          # attention splits: scratch in use
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    lat, out_a = _frames(cfg, z)
+    _, out_b = _frames(cfg, z)
+    a, b = FlashDecoder(cfg, w), FlashDecoder(cfg, w)
+    try:
+        a.reset()
+        b.reset()
+        for t in range(2):                             # two calls in a row
+            a.decode_frame(lat[t], out_a[t])
+            b.decode_frame_static_scratch(lat[t], out_b[t])
+        # the handle's graph is back on its own scratch afterwards
+        a.decode_frame(lat[2], out_a[2])
+        b.decode_frame(lat[2], out_b[2])
+        torch.cuda.synchronize()
+        assert a.status() == 0 and b.status() == 0
+        for t in range(3):
+            np.testing.assert_array_equal(out_b[t].float().cpu().numpy(),
+                                          out_a[t].float().cpu().numpy())
+    finally:
+        a.close()
+        b.close()
+
+
+def test_handle_without_splitting_runs_the_plain_step():
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder
+    cfg = small_bf16(attn_splits=1, frames=2)
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    lat, out_a = _frames(cfg, z)
+    _, out_b = _frames(cfg, z)
+    a, b = FlashDecoder(cfg, w), FlashDecoder(cfg, w)
+    try:
+        a.reset()
+        b.reset()
+        for t in range(2):
+            a.decode_frame(lat[t], out_a[t])
+            b.decode_frame_static_scratch(lat[t], out_b[t])
+        torch.cuda.synchronize()
+        for t in range(2):
+            np.testing.assert_array_equal(out_b[t].float().cpu().numpy(),
+                                          out_a[t].float().cpu().numpy())
+    finally:
+        a.close()
+        b.close()
+
+
+def test_oversize_scratch_is_refused():
+    import torch
+    from streaming_transformer_video_b200 import FlashDecoder, flashdec as fdb
+    # 13 query tiles x 16 heads x 4 splits x 33 KB = 27 MB > the fixed 8 MiB
+    cfg = fd_synth.CONFIGS["480p_wan21"].replace(attn_splits=4)
+    w = fd_synth.make_weights(cfg)
+    dec = FlashDecoder(cfg, w)
+    try:
+        dec.reset()
+        lat = torch.zeros((cfg.latent_ch, cfg.grid_h, cfg.grid_w), dtype=torch.bfloat16, device="cuda")
+        out = torch.empty(cfg.out_shape, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(fdb.FDError) as e:
+            dec.decode_frame_static_scratch(lat, out)
+        assert e.value.code == fdb.FD_ERR_UNSUPPORTED
+        assert dec.frame_index() == 0                  # nothing was enqueued
+    finally:
+        dec.close()
