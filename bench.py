@@ -40,8 +40,8 @@ DEFAULT_CONFIG = "1080p_wan22"
 # profiles/block_1080p_ncu_full.md. Keyed by the sha256 of the kernel source:
 # when the kernel changes the figure no longer applies and is reported as null.
 NCU_ATTN_TRAFFIC = {
-    ("1080p_wan22", "57eedbc751f7f407cadbe0cf1292d601e65ddbdfa8315696fefbda8e5e8c64da"):
-        117092864 + 9040128,
+    ("1080p_wan22", "97cf5174fe98f8189f7652838c6f3553b8488c727c340500335f57fb58ff6c60"):
+        164032512 + 57520384,
 }
 
 
