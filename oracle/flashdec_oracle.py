@@ -31,14 +31,13 @@ notes of the repository):
   * FP8 MLP ([FD] Sec. 4.6, "static-calibrated FP8 quantization of all MLP
     layers"): the MLP sublayer of every Transformer block (backbone and
     refinement; not the pixel head's spatial MLP) multiplies E4M3 operands.
-    Per-tensor static scales: each weight matrix s_w = max|W| / 448; the
-    activations entering each Linear have a scale fixed by calibration
-    (max |activation| over calibration frames / 448). The first Linear's
-    operand is the residual stream x itself: the RMSNorm gain is folded into
-    W_1 before W_1 is quantized and the RMSNorm row scale multiplies the
-    product, so only the point where the rounding happens differs from
-    quantizing the normalised input. The hidden activation is quantized
-    after GELU. Rounding: nearest, ties to even, saturating at +-448.
+    Each of its two Linear layers quantizes exactly what it multiplies: its
+    input activation and its weight matrix. The first Linear's input is the
+    RMSNorm output a = x / rms(x) * g (gain included); the second's is the
+    GELU output h. Per-tensor static scales: each weight matrix s_w =
+    max|W| / 448; each activation a scale fixed by calibration (max |a| and
+    max |h| over calibration frames through the unquantized decoder, / 448).
+    Rounding: nearest, ties to even, saturating at +-448.
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py
 (library routines, closed forms, invariants of the method). No function
@@ -153,27 +152,24 @@ def mlp(cfg, w: Dict[str, np.ndarray], p: str, x: np.ndarray,
     """Pre-norm MLP sublayer of block p (without the residual add):
     GELU(RMSNorm(x) W_1^T + b_1) W_2^T + b_2 ([FD] Sec. 3.2).
 
-    With cfg.mlp_fp8 the two Linears multiply FP8 operands with static
-    per-tensor scales w[p + "fp8_sx"] (x) and w[p + "fp8_sh"] (hidden):
-      r  = 1 / sqrt(mean(x^2) + eps)                 per token
-      W1g = W_1 diag(g)       quantized with its own scale
-      h  = GELU(r (Q(x) W1g_q^T) + b_1)
-      y  = Q(h) W2_q^T + b_2
-    amax (calibration, unquantized MLP only): records the largest |x| and
-    |h| of the block under keys p + "x" and p + "h"."""
-    g = w[p + "norm2_g"]
+    With cfg.mlp_fp8 each Linear multiplies the FP8 images of its own input
+    and weight ([FD] Sec. 4.6), with static per-tensor scales
+    w[p + "fp8_sa"] (the normalised input a) and w[p + "fp8_sh"] (hidden h):
+      a  = RMSNorm(x) (gain g included)
+      h  = GELU(Q(a) Q(W_1)^T + b_1)
+      y  = Q(h) Q(W_2)^T + b_2
+    amax (calibration, unquantized MLP only): records the largest |a| and
+    |h| of the block under keys p + "a" and p + "h"."""
+    a = rms_norm(x, w[p + "norm2_g"], cfg.norm_eps)
     if not getattr(cfg, "mlp_fp8", 0):
-        a = rms_norm(x, g, cfg.norm_eps)
         h = gelu(linear(a, w[p + "w1"], w[p + "b1"]))
         if amax is not None:
-            amax[p + "x"] = max(amax.get(p + "x", 0.0), float(np.max(np.abs(x))))
+            amax[p + "a"] = max(amax.get(p + "a", 0.0), float(np.max(np.abs(a))))
             amax[p + "h"] = max(amax.get(p + "h", 0.0), float(np.max(np.abs(h))))
         return linear(h, w[p + "w2"], w[p + "b2"])
-    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + cfg.norm_eps)
-    w1g = w[p + "w1"] * g[None, :]
-    w1q = quantize_weight(w1g, weight_scale(w1g))
+    w1q = quantize_weight(w[p + "w1"], weight_scale(w[p + "w1"]))
     w2q = quantize_weight(w[p + "w2"], weight_scale(w[p + "w2"]))
-    h = gelu(r * (quantize_act(x, float(w[p + "fp8_sx"])) @ w1q.T) + w[p + "b1"])
+    h = gelu(quantize_act(a, float(w[p + "fp8_sa"])) @ w1q.T + w[p + "b1"])
     return quantize_act(h, float(w[p + "fp8_sh"])) @ w2q.T + w[p + "b2"]
 
 
@@ -370,14 +366,27 @@ class OracleDecoder:
         frames = self.window_frames(l)
         return self.cache[l][frames.index(frame)]
 
+    def refine_window(self, l: int):
+        """Paper head: sub-frame indices t r_t + tau held by refinement block
+        l's cache, oldest first."""
+        n = len(self.rcache[l])
+        end = self.t * self.cfg.r_t
+        return list(range(end - n, end))
+
+    def refine_cached_kv(self, l: int, sub: int):
+        """Un-rotated (k, v) [L_frm][G][D_h] of sub-frame `sub` in refinement
+        block l's cache."""
+        return self.rcache[l][self.refine_window(l).index(sub)]
+
 
 def calibrate_fp8(cfg, weights, z: np.ndarray) -> Dict[str, float]:
     """Static FP8 scales of every MLP layer ([FD] Sec. 4.6: static
     calibration): stream the calibration frames z[0..T-1] through the decoder
-    with unquantized MLPs, take per block the largest |x| entering the MLP and
-    the largest |GELU output|, and set each scale to fp32(amax / 448), so the
-    calibration data never saturates. Returns {"b{l}.fp8_sx": s, "b{l}.fp8_sh":
-    s, ...}, with "r{l}.*" for the paper head's refinement blocks."""
+    with unquantized MLPs, take per block the largest |a| entering the first
+    MLP Linear (the RMSNorm output) and the largest |GELU output|, and set each
+    scale to fp32(amax / 448), so the calibration data never saturates.
+    Returns {"b{l}.fp8_sa": s, "b{l}.fp8_sh": s, ...}, with "r{l}.*" for the
+    paper head's refinement blocks."""
     dec = OracleDecoder(cfg.replace(mlp_fp8=0), weights)
     dec.amax = {}
     for t in range(z.shape[0]):

@@ -101,7 +101,7 @@ def test_fp8_paper_head_matches_torch_library_composition():
     w = fd_synth.make_weights(cfg)
     z = fd_synth.make_latents(cfg, frames=4)
     scales = oracle.calibrate_fp8(cfg, w, z)
-    assert set(scales) == {f"{p}fp8_s{k}" for p in ("b0.", "r0.", "r1.") for k in "xh"}
+    assert set(scales) == {f"{p}fp8_s{k}" for p in ("b0.", "r0.", "r1.") for k in "ah"}
     cfg8, w8 = cfg.replace(mlp_fp8=1), {**w, **scales}
     got = oracle.decode_video(cfg8, w8, z)
     np.testing.assert_allclose(got, _torch_library_paper_decoder(cfg8, w8, z), rtol=1e-9, atol=1e-9)
@@ -114,7 +114,7 @@ def test_calibration_is_the_amax_of_the_unquantized_mlp_activations():
     scales = oracle.calibrate_fp8(cfg, w, z)
     amax = {}
     _torch_library_decoder(cfg, w, z, amax)               # one pass over all frames
-    assert set(scales) == {f"b{l}.fp8_s{k}" for l in range(cfg.n_blocks) for k in "xh"}
+    assert set(scales) == {f"b{l}.fp8_s{k}" for l in range(cfg.n_blocks) for k in "ah"}
     for key, a in amax.items():
         p, kind = key[:-1], key[-1]
         assert scales[p + "fp8_s" + kind] == float(np.float32(a / 448.0))

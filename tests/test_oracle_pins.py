@@ -173,22 +173,23 @@ def test_rope_3d_parts_follow_their_own_axis():
 def _torch_f8(t, s):
     """Dequantized FP8 E4M3 value of t with scale s through torch's own
     float8_e4m3fn cast (its rounding is an implementation independent of the
-    oracle's); the quotient is formed in float32, values must stay below 464
-    (torch turns larger ones into NaN instead of saturating)."""
+    oracle's); the quotient is formed in float32. torch's cast turns values of
+    464 and more into NaN instead of saturating, so they are first clamped to
+    the largest finite value 448 (the format's saturating conversion)."""
     q = (t.float() * torch.tensor(1.0 / float(s), dtype=torch.float64).float())
-    return q.to(torch.float8_e4m3fn).double() * float(s)
+    return q.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).double() * float(s)
 
 
 def _torch_mlp(cfg, W, p, x, amax=None):
-    """MLP sublayer from torch calls; with cfg.mlp_fp8 the operands of both
-    Linears are FP8 (weights: per-tensor scale max|w|/448 in float32, the
-    RMSNorm gain folded into W_1 first; activations: the static scales)."""
-    g = W[p + "norm2_g"]
+    """MLP sublayer from torch calls; with cfg.mlp_fp8 each Linear multiplies
+    FP8 images of its own input and weight (weights: per-tensor scale
+    max|w|/448 in float32; activations a = RMSNorm(x) and h: the static
+    scales)."""
+    a = F.rms_norm(x, (cfg.d_model,), W[p + "norm2_g"], eps=cfg.norm_eps)
     if not getattr(cfg, "mlp_fp8", 0):
-        a = F.rms_norm(x, (cfg.d_model,), g, eps=cfg.norm_eps)
         h = F.gelu(F.linear(a, W[p + "w1"], W[p + "b1"]))
         if amax is not None:
-            amax[p + "x"] = max(amax.get(p + "x", 0.0), float(x.abs().max()))
+            amax[p + "a"] = max(amax.get(p + "a", 0.0), float(a.abs().max()))
             amax[p + "h"] = max(amax.get(p + "h", 0.0), float(h.abs().max()))
         return F.linear(h, W[p + "w2"], W[p + "b2"])
 
@@ -196,8 +197,7 @@ def _torch_mlp(cfg, W, p, x, amax=None):
         s = float(torch.tensor(float(w.abs().max()) / 448.0).float())
         return (w / s).to(torch.float8_e4m3fn).double() * s
 
-    r = torch.rsqrt((x * x).mean(-1, keepdim=True) + cfg.norm_eps)
-    h = F.gelu(r * F.linear(_torch_f8(x, W[p + "fp8_sx"]), wq(W[p + "w1"] * g)) + W[p + "b1"])
+    h = F.gelu(F.linear(_torch_f8(a, W[p + "fp8_sa"]), wq(W[p + "w1"]), W[p + "b1"]))
     return F.linear(_torch_f8(h, W[p + "fp8_sh"]), wq(W[p + "w2"]), W[p + "b2"])
 
 
