@@ -92,9 +92,10 @@ def kind_flops(cfg):
 
 
 def kernels_per_frame(cfg) -> int:
-    n = 2 + 5 * cfg.n_blocks                            # step_begin, embed, backbone
+    per_block = 5 + (1 if getattr(cfg, "mlp_fp8", 0) else 0)   # FP8: + MLP-input quantization
+    n = 2 + per_block * cfg.n_blocks                    # step_begin, embed, backbone
     if is_paper(cfg):
-        return n + 1 + cfg.r_t * (5 * cfg.n_refine + 2)  # upsample, refinement, spatial MLP
+        return n + 1 + cfg.r_t * (per_block * cfg.n_refine + 2)  # upsample, refinement, spatial MLP
     return n + 1                                        # final
 
 

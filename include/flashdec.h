@@ -52,7 +52,12 @@ typedef enum {
   FD_ERR_OOM = -3,           /* device allocation failed                      */
   FD_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed             */
   FD_ERR_TIMEOUT = -5,       /* a device-side wait ran out (see fd_status)    */
-  FD_ERR_BAD_HANDLE = -6     /* null, destroyed or foreign handle             */
+  FD_ERR_BAD_HANDLE = -6,    /* null, destroyed or foreign handle             */
+  FD_ERR_BOUNDS = -7         /* bounds-checked build only (libflashdec_debug.so):
+                                a kernel computed a ring row, slot, V^T column,
+                                split-partial index or pixel offset outside its
+                                buffer, skipped that access and recorded this
+                                code (see fd_status)                          */
 } fd_status_t;
 
 typedef enum { FD_F32 = 0, FD_BF16 = 1 } fd_dtype;
@@ -94,13 +99,18 @@ typedef struct {
                             refinement) multiplies FP8 E4M3 operands with static
                             per-tensor scales (Sec. 4.6, optimization 4). Needs
                             dtype BF16, d_model a multiple of 128 and
-                            fd_weights.mlp_scales. Weights are quantized here:
-                            W_1 diag(norm2_g) and W_2 each with the scale
-                            fp32(max|W| / 448), round to nearest even        */
-  int32_t record_mlp_amax; /* 1 (mlp_fp8 = 0 only): the MLP epilogues record,
-                            per block, max |x| entering the MLP and max |GELU
-                            output| since the last fd_reset; read them as
-                            static scales with fd_mlp_fp8_scales             */
+                            fd_weights.mlp_scales. Each MLP Linear multiplies
+                            the E4M3 images of its own input and weight: W_1
+                            and W_2 are quantized here, each with the scale
+                            fp32(max|W| / 448), round to nearest even; the
+                            first Linear's input RMSNorm(x) (gain included)
+                            and the second's input GELU(..) with the static
+                            scales of fd_weights.mlp_scales                */
+  int32_t record_mlp_amax; /* 1 (mlp_fp8 = 0 only; d_model a multiple of 128):
+                            record, per block, max |RMSNorm(x)| entering the
+                            MLP and max |GELU output| since the last fd_reset;
+                            read them as static scales with
+                            fd_mlp_fp8_scales                               */
   int32_t batch;         /* B video streams decoded together (1 .. 64): every
                             call takes one latent frame of each stream; each
                             stream has its own frame counter and ring slots
@@ -135,12 +145,11 @@ typedef struct {
  *   out_w [C P^2][D], out_b [C P^2]     second layer, channel order (c, dy, dx)
  * (up_w .. sp1_b are ignored with head_mode 0.)
  * With mlp_fp8 = 1:
- *   mlp_scales[l] -> 2 floats {s_x, s_h}, one entry per block (backbone, then
- *            refinement): static scales of the MLP input x and of the GELU
- *            output h. x is stored as e4m3(x / s_x) before the RMSNorm row scale
- *            (which, like the gain, multiplies the fp32 product), h as
- *            e4m3(h / s_h); rounding to nearest even, saturating at +-448.
- *            Ignored with mlp_fp8 = 0.
+ *   mlp_scales[l] -> 2 floats {s_a, s_h}, one entry per block (backbone, then
+ *            refinement): static scales of the inputs of the two MLP Linears,
+ *            a = RMSNorm(x) (with gain norm2_g) and the GELU output h, stored
+ *            as e4m3(a / s_a) and e4m3(h / s_h); rounding to nearest even,
+ *            saturating at +-448. Ignored with mlp_fp8 = 0.
  */
 typedef struct {
   const float *embed_w, *embed_b;
@@ -197,10 +206,16 @@ FD_API fd_status_t fd_decode_frame(fd_handle* h, const void* latent_frame, void*
 
 /*
  * Same as fd_decode_frame with HOST buffers: copies the latent frame to the
- * device, decodes it and copies the pixels back, all on `stream`.
- * For truly asynchronous copies both buffers should be pinned
- * (cudaHostAlloc / cudaHostRegister). `out_pixels` is complete once the
- * stream has been synchronised.
+ * device, decodes it and copies the pixels back. `out_pixels` is complete
+ * once `stream` has been synchronised. The copy-out runs on `stream`; the
+ * copy-in and the frame's graph run on a stream of the handle, after all work
+ * enqueued on `stream` before this call and after the copy-out of two frames
+ * earlier (two device staging slots, used in turn). So the copy-out of frame
+ * t overlaps the decode of frame t+1 when the caller does not synchronise in
+ * between. Results are bit-identical to fd_decode_frame. For truly
+ * asynchronous copies both buffers should be pinned (cudaHostAlloc /
+ * cudaHostRegister), and each out_pixels buffer must stay untouched until
+ * its copy-out has completed.
  */
 FD_API fd_status_t fd_decode_frame_host(fd_handle* h, const void* latent_frame_host,
                                  void* out_pixels_host, void* stream);
@@ -243,13 +258,51 @@ FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
 
 /*
+ * Test/debug: copy ring slot `slot` of block `block`, video stream b
+ * (0 <= b < batch), to host memory as fp32 [G][L_frm][D_h]. Blocks
+ * 0 .. n_blocks-1 are the backbone (slots 0 .. W); with head_mode 1, blocks
+ * n_blocks .. n_blocks + n_refine - 1 are the refinement blocks, whose ring
+ * holds r_t (W+1) sub-frames (sub-frame s in slot s mod r_t (W+1), [FD]
+ * Sec. 3.4 Step 2). kv as for fd_debug_read_slot. Synchronous.
+ */
+FD_API fd_status_t fd_debug_read_ring(fd_handle* h, int block, int b, int slot, int kv,
+                                      float* host_dst);
+
+/*
+ * Test/debug: fill device state with values that must never reach an output,
+ * enqueued on `stream`. FD_POISON_RING sets every byte of the ring caches
+ * (backbone and refinement) to 0xFF, a NaN in bf16 and fp32: a decode after
+ * fd_reset + this call must give the same outputs as after fd_reset alone,
+ * because a frame only reads ring slots written since the reset ([FD] Sec. 3.3:
+ * the cache holds only frames that exist). FD_POISON_SPLIT_COUNTERS sets the
+ * attention key-splitting counters to 0x7F7F7F7F, which breaks the handle's own
+ * split combine until the next fd_reset (a positive control for the fixed-
+ * scratch entry point below).
+ */
+enum { FD_POISON_RING = 1, FD_POISON_SPLIT_COUNTERS = 2 };
+FD_API fd_status_t fd_debug_poison(fd_handle* h, int32_t what, void* stream);
+
+/*
+ * Test/debug: set stream b's frame counter to t (>= 0), so that the next
+ * decoded frame is treated as frame t (ring slot t mod (W+1), temporal RoPE
+ * at index t); nothing else changes. Lets a test reach very long videos
+ * ([FD] Sec. 4.3 "Long Video Decoding": length is unbounded) without decoding
+ * every frame before them: once n_blocks W + 1 frames have been decoded after
+ * the jump, every slot that frame t reads was written after it, so the output
+ * equals that of a video that really started at frame 0 (positions enter the
+ * attention only through differences). Synchronous on `stream`.
+ */
+FD_API fd_status_t fd_debug_set_frame_index(fd_handle* h, int b, int64_t t, void* stream);
+
+/*
  * Test/debug: run the second half of block `block` (backbone blocks first,
  * then refinement blocks) once on a given residual stream: x_host becomes
  * the stream, the attention output is set to zero, and the
- * block's O-projection (so x + b_o), MLP-up and MLP-down kernels run with
- * the handle's weights (FP8 with mlp_fp8); the resulting stream
- * x + b_o + MLP(x + b_o) is copied to out_host. Both are [batch L_frm][D] fp32. Both sides of
- * a parity test then quantize identical float32 inputs. Synchronous;
+ * block's O-projection (so x + b_o), MLP-up and MLP-down kernels (with
+ * mlp_fp8 the E4M3 quantization of RMSNorm(x + b_o) in between) run with the
+ * handle's weights; the resulting stream x + b_o + MLP(x + b_o) is copied to
+ * out_host. Both are [batch L_frm][D] fp32. Both sides of a parity test then
+ * start the MLP from identical float32 values. Synchronous;
  * overwrites the handle's per-frame scratch (not the ring cache), so it must
  * not overlap a decode; records no calibration ranges.
  */
@@ -270,7 +323,9 @@ FD_API fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_ho
 typedef enum {
   FD_K_STEP_BEGIN = 0, FD_K_EMBED = 1, FD_K_QKV = 2, FD_K_ATTN = 3,
   FD_K_OPROJ = 4, FD_K_MLP_UP = 5, FD_K_MLP_DOWN = 6, FD_K_FINAL = 7,
-  FD_K_UPSAMPLE = 8, FD_K_SPATIAL = 9
+  FD_K_UPSAMPLE = 8, FD_K_SPATIAL = 9,
+  FD_K_MLP_NORM = 10   /* mlp_fp8: RMSNorm + E4M3 quantization of the MLP input
+                          (after each O-projection); record_mlp_amax: its range */
 } fd_kernel_kind;
 FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* kind_out,
                                    int32_t cap, int32_t* n_out);
@@ -278,23 +333,33 @@ FD_API fd_status_t fd_last_step_kernel_ms(fd_handle* h, float* ms_out, int32_t* 
 /*
  * fd_decode_frame without the handle's attention scratch (the paper has no
  * counterpart: this is a deployment variant of this library). Identical
- * results to fd_decode_frame. When the handle's attention splits its key
- * ranges (fd_config.attn_splits, or the automatic choice), the partial
- * results and counters of that split live in one fixed, statically sized
- * device array of this library (8 MiB) instead of memory allocated by
- * fd_create; this call allocates nothing. Handles whose split needs more than
- * 8 MiB ((L/128 rounded up) x heads x batch x splits x 33 KB, plus 4 bytes per
- * unit) get FD_ERR_UNSUPPORTED; handles that do not split simply run
- * fd_decode_frame.
+ * results to fd_decode_frame. Some callers cannot allocate device memory at
+ * the point where they decode: code running inside a host that pre-plans all
+ * of its memory (an inference server's memory pool or a pre-allocated arena),
+ * or that must not call cudaMalloc between two frames because it would
+ * synchronise the device and break a frame's latency budget. When the
+ * handle's attention splits its key ranges (fd_config.attn_splits, or the
+ * automatic choice), the partial results and counters of that split live in
+ * one fixed, statically sized device array of this library (8 MiB) instead of
+ * memory allocated by fd_create; this call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine). Handles whose split needs more
+ * than the array (64 KiB of counters, then (L/128 rounded up) x heads x batch
+ * x splits x 33 KB of partials) get FD_ERR_UNSUPPORTED; handles that do not
+ * split simply run fd_decode_frame.
  *  - The array is shared by every handle and stream of the process on that
- *    device: calls that overlap in time (different streams, threads or
- *    handles, or an fd_decode_frame_static_scratch still running on the GPU
- *    when another is enqueued on a different stream) race on it and give wrong
- *    results. Serialise them on one stream.
- *  - The first call on each device resolves the array's address
- *    (cudaGetSymbolAddress); make it outside any CUDA stream capture. Each
- *    call also updates the attention nodes of the handle's frame graph before
- *    and after enqueueing it, so it must not be captured either.
+ *    device and keeps the last call's contents. Each call first clears the
+ *    counters it uses (an enqueued memset, no allocation), so serialised calls
+ *    of different handles are independent. Calls that overlap in time
+ *    (different streams, threads or handles, or an
+ *    fd_decode_frame_static_scratch still running on the GPU when another is
+ *    enqueued on a different stream) race on it and give wrong results.
+ *    Serialise them on one stream.
+ *  - The current device must be the one the handle was created on
+ *    (FD_ERR_INVALID_ARG otherwise). The first call on each device resolves
+ *    the array's address there (cudaGetSymbolAddress); make that first call
+ *    outside any CUDA stream capture. Each call also updates the attention
+ *    nodes of the handle's frame graph before and after enqueueing it, and
+ *    puts them back on the handle's own scratch even when it fails.
  * Errors as for fd_decode_frame, plus FD_ERR_UNSUPPORTED for oversize.
  */
 FD_API fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent_frame,
@@ -303,7 +368,7 @@ FD_API fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* late
 /*
  * Static FP8 scales from the calibration recorded by a handle created with
  * record_mlp_amax = 1 ([FD] Sec. 4.6: static calibration): for every block
- * (backbone, then refinement), scales_out[2 l] = fp32(max |x| / 448) and
+ * (backbone, then refinement), scales_out[2 l] = fp32(max |RMSNorm(x)| / 448) and
  * scales_out[2 l + 1] = fp32(max |h| / 448) over the frames decoded since the
  * last fd_reset (1 where nothing was seen), ready for fd_weights.mlp_scales of
  * an mlp_fp8 handle. *n_out = 2 * (n_blocks + n_refine); cap = 0 queries it.

@@ -62,6 +62,14 @@ fd_status_t fail(fd_status_t s, const char* fmt, ...) {
     if (s_ != FD_OK) return s_;          \
   } while (0)
 
+// Consecutive kernels of the frame graph are linked by programmatic edges
+// (programmatic dependent launch; every kernel orders its data accesses with
+// griddep_wait). Builds with -DFD_PDL=0 use full dependencies instead.
+#ifndef FD_PDL
+#define FD_PDL 1
+#endif
+constexpr bool kUsePdl = FD_PDL != 0;
+
 constexpr uint32_t kMagic = 0xFDEC0DE5u;
 constexpr uint32_t kDead = 0xDEADFD00u;
 
@@ -210,6 +218,7 @@ struct fd_handle {
   int* split_ctr = nullptr;
   int fs_stride = 1;                // FrameStates per stream: 1 (+ r_t, paper head)
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
+  int device = -1;                  // the CUDA device the handle was created on
   int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
   size_t k_bytes = 0, v_bytes = 0, rk_bytes = 0, rv_bytes = 0;
   size_t latent_elems = 0, out_elems = 0, io_elt = 0, elt = 0;
@@ -227,8 +236,11 @@ struct fd_handle {
   void *kc = nullptr, *vtc = nullptr;
   void *rkc = nullptr, *rvtc = nullptr;     // refinement ring (paper head)
   // FP8 MLP: per block (backbone, then refinement) static activation scales
-  // and per-tensor weight scales; x8 = E4M3 copy of x for the MLP-up
-  std::vector<float> s_x, s_h, s_w1, s_w2;
+  // and per-tensor weight scales; x8 = E4M3 image of the MLP-up's input
+  // RMSNorm(x) / s_a; g2 = the RMSNorm gains before the MLP (fp32, also kept
+  // for calibration, which records max |RMSNorm(x)|)
+  std::vector<float> s_a, s_h, s_w1, s_w2;
+  std::vector<float*> g2;
   void* x8 = nullptr;
   unsigned* amax = nullptr;                 // calibration: [blocks][2] float bits
   int n_amax = 0;
@@ -237,10 +249,22 @@ struct fd_handle {
   void* xsb = nullptr;                      // [r_t][M][D] storage type
   void *xb = nullptr, *q = nullptr, *o = nullptr, *hb = nullptr;
   float2 *rope_row = nullptr, *rope_col = nullptr;
+  double* inv_freq_t = nullptr;             // temporal RoPE frequencies theta^(-2m/d_t)
   long long* ctr = nullptr;
   FrameState* fs = nullptr;
   int* status = nullptr;
-  void *latent_stage = nullptr, *out_stage = nullptr;
+  // fd_decode_frame_host: two staging slots, so that the copy-out of frame t
+  // (on the caller's stream) runs under the graph of frame t+1 (on host_stream)
+  void* latent_stage[2] = {nullptr, nullptr};
+  void* out_stage[2] = {nullptr, nullptr};
+  cudaStream_t host_stream = nullptr;
+  cudaEvent_t ev_graph[2] = {nullptr, nullptr};   // graph of the slot's frame done
+  cudaEvent_t ev_d2h[2] = {nullptr, nullptr};     // copy-out of the slot's frame done
+  cudaEvent_t ev_user = nullptr;                   // caller-stream work before a host call
+  bool d2h_pending[2] = {false, false};
+  int host_slot = 0;
+  int g_last = -1;          // slot of the last graph on host_stream not yet joined
+  bool user_pending = true; // caller-stream work since the last host call
 
   // TMA maps (bf16 path)
   CUtensorMap tm_xb{}, tm_o{}, tm_h{}, tm_q{}, tm_k{}, tm_v{}, tm_wout{};
@@ -251,6 +275,7 @@ struct fd_handle {
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
   cudaGraphNode_t last_node = nullptr;
+  bool last_is_kernel = false;
   cudaGraphNode_t embed_node = nullptr;
   KernelLaunch embed_launch{};
   EmbedParams embed_p{};
@@ -328,6 +353,12 @@ struct fd_handle {
     if (exec) cudaGraphExecDestroy(exec);
     if (graph) cudaGraphDestroy(graph);
     for (auto e : events) cudaEventDestroy(e);
+    for (int i = 0; i < 2; ++i) {
+      if (ev_graph[i]) cudaEventDestroy(ev_graph[i]);
+      if (ev_d2h[i]) cudaEventDestroy(ev_d2h[i]);
+    }
+    if (ev_user) cudaEventDestroy(ev_user);
+    if (host_stream) cudaStreamDestroy(host_stream);
     for (void* p : allocs) cudaFree(p);
   }
 
@@ -340,6 +371,7 @@ struct fd_handle {
     FD_CUDA(cudaGraphAddEventRecordNode(&n, graph, last_node ? &last_node : nullptr,
                                         last_node ? 1 : 0, ev));
     last_node = n;
+    last_is_kernel = false;
     return FD_OK;
   }
   // kernel_timing 1: one event after every kernel (consecutive events bracket
@@ -358,9 +390,20 @@ struct fd_handle {
     np.sharedMemBytes = unsigned(k.smem);
     np.kernelParams = args;
     cudaGraphNode_t n;
-    FD_CUDA(cudaGraphAddKernelNode(&n, graph, last_node ? &last_node : nullptr, last_node ? 1 : 0,
-                                   &np));
+    if (last_node && last_is_kernel && kUsePdl) {
+      // programmatic edge: this kernel may launch once every CTA of the
+      // previous one has started; its griddep_wait() orders the data
+      FD_CUDA(cudaGraphAddKernelNode(&n, graph, nullptr, 0, &np));
+      cudaGraphEdgeData edge{};
+      edge.from_port = cudaGraphKernelNodePortProgrammatic;
+      edge.type = cudaGraphDependencyTypeProgrammatic;
+      FD_CUDA(cudaGraphAddDependencies_v2(graph, &last_node, &n, &edge, 1));
+    } else {
+      FD_CUDA(cudaGraphAddKernelNode(&n, graph, last_node ? &last_node : nullptr,
+                                     last_node ? 1 : 0, &np));
+    }
     last_node = n;
+    last_is_kernel = true;
     if (out_node) *out_node = n;
     kinds.push_back(k.kind);
     if (cfg.kernel_timing == 1 || bracket) {
@@ -377,6 +420,7 @@ struct fd_handle {
   fd_status_t add_out_gemm(OutNode on, int N);
   fd_status_t add_block(int wi, const BlockIO& io);
   fd_status_t add_post_attention(int wi, const BlockIO& io);
+  fd_status_t add_norm_quant(const BlockIO& io, int wi, float q_inv, unsigned* rec);
   EpiParams base_epi(const BlockIO& io) const;
   size_t split_units() const { return size_t((L + 127) / 128) * cfg.n_heads * B; }
   BlockIO backbone_io(int layer);
@@ -471,6 +515,9 @@ EpiParams fd_handle::base_epi(const BlockIO& io) const {
   e.pl_add = 0;
   e.acc_scale = 1.f;
   e.q_inv = 1.f;
+  e.status = status;
+  e.n_sub = cfg.r_t;
+  e.out_frames = cfg.out_ch * cfg.r_t;
   return e;
 }
 
@@ -577,6 +624,8 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(Dh)));
     ap.fs = io.fs;
     ap.status = status;
+    ap.kv_rows = io.kv_rows;
+    ap.n_slabs = (io.kv_rows == kv_rows ? cfg.n_blocks : cfg.n_refine) * B * G;
     // one 128-query tile per CTA, two CTAs per SM (measured faster than two
     // query tiles sharing one CTA, and than three CTAs with single-buffered S)
     using A = TcAttnSmem;
@@ -625,17 +674,17 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
   const int D = cfg.d_model, H = cfg.n_heads, Dh = cfg.head_dim;
   EpiParams e;
   if (fp8) {
-    // output projection + residual; x also stored as e4m3(x / s_x)
+    // output projection + residual (x32 and its sums of squares only)
     e = base_epi(io);
     e.bias = bo[wi];
-    e.x8 = x8;
-    e.q_inv = float(1.0 / double(s_x[wi]));
     FD_TRY(add_gemm(EPI_RESID_Q, FD_K_OPROJ, tm_o, o, tm_wo[wi], wo[wi], D, H * Dh, e, nullptr));
-    // FP8 MLP up: h = GELU(r (x8 W1q^T) s_x s_w1 + b_1) stored as e4m3(h / s_h)
+    // the MLP-up's input: x8 = e4m3(RMSNorm(x) / s_a)
+    FD_TRY(add_norm_quant(io, wi, float(1.0 / double(s_a[wi])), nullptr));
+    // FP8 MLP up: h = GELU((x8 W1q^T) s_a s_w1 + b_1) stored as e4m3(h / s_h)
     e = base_epi(io);
     e.bias = b1[wi];
     e.hout = hb;
-    e.acc_scale = float(double(s_x[wi]) * double(s_w1[wi]));
+    e.acc_scale = float(double(s_a[wi]) * double(s_w1[wi]));
     e.q_inv = float(1.0 / double(s_h[wi]));
     FD_TRY(add_gemm(EPI_GELU_Q, FD_K_MLP_UP, tm_x8, x8, tm_w1[wi], w1[wi], dff, D, e, nullptr,
                     true));
@@ -649,9 +698,10 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
   // output projection + residual
   e = base_epi(io);
   e.bias = bo[wi];
-  if (amax) e.amax = amax + 2 * wi;               // calibration: max |x| entering the MLP
   FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[wi] : tm_o, wo[wi], D, H * Dh, e,
                   nullptr));
+  // calibration: max |RMSNorm(x)| entering the MLP
+  if (amax) FD_TRY(add_norm_quant(io, wi, 1.f, amax + 2 * wi));
   // MLP up + GELU
   e = base_epi(io);
   e.bias = b1[wi];
@@ -666,25 +716,46 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
                   nullptr);
 }
 
+// RMSNorm(x) of the MLP's input (gain of block wi): its E4M3 image
+// e4m3(a q_inv) into x8 (FP8 MLP), or with rec set its max |a| (calibration).
+fd_status_t fd_handle::add_norm_quant(const BlockIO& io, int wi, float q_inv, unsigned* rec) {
+  NormQuantParams np{};
+  np.x32 = io.x32;
+  np.ssq = io.ssq;
+  np.g = g2[wi];
+  np.x8 = rec ? nullptr : static_cast<uint8_t*>(x8);
+  np.amax = rec;
+  np.M = M;
+  np.D = cfg.d_model;
+  np.inv_d = 1.f / float(cfg.d_model);
+  np.eps = cfg.norm_eps;
+  np.q_inv = q_inv;
+  KernelLaunch k{reinterpret_cast<const void*>(&mlp_norm_quant_kernel), dim3((M + 7) / 8),
+                 dim3(256), 0, FD_K_MLP_NORM};
+  void* args[] = {&np};
+  return add_kernel(k, args);
+}
+
 fd_status_t fd_handle::build_graph() {
   FD_CUDA(cudaGraphCreate(&graph, 0));
   last_node = nullptr;
+  last_is_kernel = false;
   if (cfg.kernel_timing == 1) FD_TRY(add_event());
 
   // step_begin
   {
-    KernelLaunch k{reinterpret_cast<const void*>(&step_begin_kernel), dim3(1), dim3(32), 0,
+    KernelLaunch k{reinterpret_cast<const void*>(&step_begin_kernel), dim3(1), dim3(256), 0,
                    FD_K_STEP_BEGIN};
     long long* c = ctr;
     FrameState* f = fs;
-    int W = cfg.window, dh = cfg.head_dim, n_sub = paper ? cfg.r_t : 0, nb = B;
-    float th = cfg.rope_theta;
-    void* args[] = {&c, &f, &W, &dh, &th, &n_sub, &nb};
+    int W = cfg.window, pairs = cfg.head_dim / 8, n_sub = paper ? cfg.r_t : 0, nb = B;
+    const double* fr = inv_freq_t;
+    void* args[] = {&c, &f, &W, &pairs, &fr, &n_sub, &nb};
     FD_TRY(add_kernel(k, args));
   }
   // embed
   {
-    embed_p.latent = latent_stage;
+    embed_p.latent = latent_stage[0];
     embed_p.latent_bf16 = cfg.io_dtype == FD_BF16;
     embed_p.C = cfg.latent_ch;
     embed_p.Hl = cfg.grid_h;
@@ -700,13 +771,14 @@ fd_status_t fd_handle::build_graph() {
     embed_p.x32 = x32;
     embed_p.xb = xb;
     embed_p.ssq = ssq;
+    embed_p.status = status;
     const void* f = bf ? reinterpret_cast<const void*>(&embed_kernel<bf16>)
                        : reinterpret_cast<const void*>(&embed_kernel<float>);
     embed_launch = KernelLaunch{f, dim3((M + kEmbedTok - 1) / kEmbedTok), dim3(256),
                                 size_t(kEmbedTok) * c_in * 4, FD_K_EMBED};
     void* args[] = {&embed_p};
     FD_TRY(add_kernel(embed_launch, args, &embed_node));
-    cur_latent = latent_stage;
+    cur_latent = latent_stage[0];
   }
   const int D = cfg.d_model;
   for (int l = 0; l < cfg.n_blocks; ++l) FD_TRY(add_block(l, backbone_io(l)));
@@ -716,7 +788,7 @@ fd_status_t fd_handle::build_graph() {
     OutNode on;
     on.p = base_epi(backbone_io(0));
     on.p.bias = bout;
-    on.p.out = out_stage;
+    on.p.out = out_stage[0];
     on.tmA = tm_xb;
     on.A = xb;
     on.tmB = bf ? tm_wout : tm_xb;
@@ -749,7 +821,7 @@ fd_status_t fd_handle::build_graph() {
       on.p = base_epi(io);
       on.p.bias = bout;
       on.p.ssq = nullptr;
-      on.p.out = out_stage;
+      on.p.out = out_stage[0];
       on.p.pl_mul = cfg.r_t;
       on.p.pl_add = tau;
       on.tmA = bf ? tm_hs : tm_xb;
@@ -760,7 +832,7 @@ fd_status_t fd_handle::build_graph() {
       FD_TRY(add_out_gemm(on, c_px));
     }
   }
-  cur_out = out_stage;
+  cur_out = out_stage[0];
   FD_CUDA(cudaGraphInstantiate(&exec, graph, 0));
   return FD_OK;
 }
@@ -819,6 +891,8 @@ fd_status_t validate(const fd_config* c) {
     return fail(FD_ERR_INVALID_ARG, "config: head_mode must be 0 or 1");
   if ((c->mlp_fp8 != 0 && c->mlp_fp8 != 1) || (c->record_mlp_amax != 0 && c->record_mlp_amax != 1))
     return fail(FD_ERR_INVALID_ARG, "config: mlp_fp8 and record_mlp_amax must be 0 or 1");
+  if (c->record_mlp_amax && c->d_model % 128)
+    return fail(FD_ERR_UNSUPPORTED, "config: record_mlp_amax needs d_model a multiple of 128");
   if (c->mlp_fp8 && (c->dtype != FD_BF16 || c->d_model % 128))
     return fail(FD_ERR_UNSUPPORTED, "config: mlp_fp8 needs dtype bf16 and d_model a multiple of 128");
   if (c->mlp_fp8 && c->record_mlp_amax)
@@ -863,6 +937,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   h->out_elems = size_t(c.out_ch) * c.r_t * h->out_h * h->out_w;
   int dev = 0;
   FD_CUDA(cudaGetDevice(&dev));
+  h->device = dev;
   int major = 0;
   FD_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
   FD_CUDA(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
@@ -888,17 +963,20 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
     FD_TRY(h->upload_w(&p, w->wo[l], D, size_t(H) * Dh, nullptr)); h->wo.push_back(p);
     if (h->fp8) {
       float s1 = 1.f, s2 = 1.f;
-      FD_TRY(h->upload_w_e4m3(&p, w->w1[l], h->dff, D, w->norm2_g[l], &s1)); h->w1.push_back(p);
+      FD_TRY(h->upload_w_e4m3(&p, w->w1[l], h->dff, D, nullptr, &s1)); h->w1.push_back(p);
       FD_TRY(h->upload_w_e4m3(&p, w->w2[l], D, h->dff, nullptr, &s2)); h->w2.push_back(p);
       h->s_w1.push_back(s1);
       h->s_w2.push_back(s2);
-      h->s_x.push_back(w->mlp_scales[l][0]);
+      h->s_a.push_back(w->mlp_scales[l][0]);
       h->s_h.push_back(w->mlp_scales[l][1]);
     } else {
       FD_TRY(h->upload_w(&p, w->w1[l], h->dff, D, w->norm2_g[l])); h->w1.push_back(p);
       FD_TRY(h->upload_w(&p, w->w2[l], D, h->dff, nullptr)); h->w2.push_back(p);
     }
     float* f;
+    if (h->fp8 || c.record_mlp_amax) {
+      FD_TRY(h->upload_f32(&f, w->norm2_g[l], D)); h->g2.push_back(f);
+    }
     FD_TRY(h->upload_f32(&f, w->bqkv[l], h->qkv)); h->bqkv.push_back(f);
     FD_TRY(h->upload_f32(&f, w->bo[l], D)); h->bo.push_back(f);
     FD_TRY(h->upload_f32(&f, w->b1[l], h->dff)); h->b1.push_back(f);
@@ -976,9 +1054,26 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   FD_TRY(h->alloc(&h->ctr, size_t(h->B) * 8));
   FD_TRY(h->alloc(&h->fs, sizeof(FrameState) * h->fs_stride * h->B));
   FD_TRY(h->alloc(&h->status, 16));
-  FD_TRY(h->alloc(&h->latent_stage, round_up(h->B * h->latent_elems * h->io_elt, 256)));
-  FD_TRY(h->alloc(&h->out_stage, round_up(h->B * h->out_elems * h->io_elt, 256)));
+  for (int i = 0; i < 2; ++i) {
+    FD_TRY(h->alloc(&h->latent_stage[i], round_up(h->B * h->latent_elems * h->io_elt, 256)));
+    FD_TRY(h->alloc(&h->out_stage[i], round_up(h->B * h->out_elems * h->io_elt, 256)));
+    FD_CUDA(cudaEventCreateWithFlags(&h->ev_graph[i], cudaEventDisableTiming));
+    FD_CUDA(cudaEventCreateWithFlags(&h->ev_d2h[i], cudaEventDisableTiming));
+  }
+  FD_CUDA(cudaEventCreateWithFlags(&h->ev_user, cudaEventDisableTiming));
+  FD_CUDA(cudaStreamCreateWithFlags(&h->host_stream, cudaStreamNonBlocking));
 
+  // ---- temporal RoPE frequencies (fp64): d_t = D_h / 4 dims, pair m at
+  // theta^(-2m/d_t); the angles themselves depend on the frame counter and are
+  // formed on the device by step_begin
+  {
+    const int dt = Dh / 4;
+    std::vector<double> fr(dt / 2);
+    for (int m = 0; m < dt / 2; ++m) fr[m] = std::pow(double(c.rope_theta), -2.0 * m / dt);
+    void* p;
+    FD_TRY(h->upload(&p, fr.data(), fr.size() * sizeof(double)));
+    h->inv_freq_t = static_cast<double*>(p);
+  }
   // ---- spatial RoPE tables (fp64 angles): row part and column part,
   // d_s = 3 D_h / 8 dims each, pair m at frequency theta^(-2m/d_s)
   {
@@ -1083,6 +1178,20 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   return FD_OK;
 }
 
+// Ordering between the caller's streams and the handle's host_stream (the
+// graphs of fd_decode_frame_host run there). Every call that enqueues work on a
+// caller stream first waits for the last such graph; fd_decode_frame_host first
+// waits for the caller-stream work enqueued since the previous host call.
+fd_status_t join_user_stream(fd_handle* h, cudaStream_t s) {
+  if (h->g_last >= 0) {
+    FD_CUDA(cudaStreamWaitEvent(s, h->ev_graph[h->g_last], 0));
+    h->g_last = -1;
+  }
+  h->user_pending = true;
+  h->last_stream = s;
+  return FD_OK;
+}
+
 fd_status_t patch_io(fd_handle* h, const void* latent, void* out) {
   if (latent != h->cur_latent) {
     h->embed_p.latent = latent;
@@ -1169,6 +1278,7 @@ fd_status_t fd_create(const fd_config* cfg, const fd_weights* weights, fd_handle
 fd_status_t fd_reset(fd_handle* h, void* stream) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_reset: invalid handle");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
   FD_CUDA(cudaMemsetAsync(h->kc, 0, h->k_bytes, s));
   FD_CUDA(cudaMemsetAsync(h->vtc, 0, h->v_bytes, s));
   if (h->paper) {
@@ -1187,6 +1297,7 @@ fd_status_t fd_reset_stream(fd_handle* h, int b, void* stream) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_reset_stream: invalid handle");
   if (b < 0 || b >= h->B) return fail(FD_ERR_INVALID_ARG, "fd_reset_stream: stream %d out of range", b);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
   FD_CUDA(cudaMemsetAsync(h->ctr + b, 0, 8, s));
   h->last_stream = s;
   return FD_OK;
@@ -1215,10 +1326,10 @@ fd_status_t fd_decode_frame(fd_handle* h, const void* latent, void* out, void* s
     return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: latent_frame is not device memory");
   if (b.type != cudaMemoryTypeDevice && b.type != cudaMemoryTypeManaged)
     return fail(FD_ERR_INVALID_ARG, "fd_decode_frame: out_pixels is not device memory");
-  FD_TRY(patch_io(h, latent, out));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
+  FD_TRY(patch_io(h, latent, out));
   FD_CUDA(cudaGraphLaunch(h->exec, s));
-  h->last_stream = s;
   return FD_OK;
 }
 
@@ -1227,12 +1338,30 @@ fd_status_t fd_decode_frame_host(fd_handle* h, const void* latent_host, void* ou
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame_host: invalid handle");
   if (!latent_host || !out_host) return fail(FD_ERR_INVALID_ARG, "fd_decode_frame_host: null buffer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  FD_CUDA(cudaMemcpyAsync(h->latent_stage, latent_host, h->B * h->latent_elems * h->io_elt,
-                          cudaMemcpyHostToDevice, s));
-  FD_TRY(patch_io(h, h->latent_stage, h->out_stage));
-  FD_CUDA(cudaGraphLaunch(h->exec, s));
-  FD_CUDA(cudaMemcpyAsync(out_host, h->out_stage, h->B * h->out_elems * h->io_elt,
+  cudaStream_t g = h->host_stream;
+  const int slot = h->host_slot;
+  // the graph runs after the caller's earlier work (a reset, a device-buffer
+  // decode) and after the copy-out that last read this slot's pixels
+  if (h->user_pending) {
+    FD_CUDA(cudaEventRecord(h->ev_user, h->last_stream));
+    FD_CUDA(cudaStreamWaitEvent(g, h->ev_user, 0));
+    h->user_pending = false;
+  }
+  if (h->d2h_pending[slot]) FD_CUDA(cudaStreamWaitEvent(g, h->ev_d2h[slot], 0));
+  FD_CUDA(cudaMemcpyAsync(h->latent_stage[slot], latent_host, h->B * h->latent_elems * h->io_elt,
+                          cudaMemcpyHostToDevice, g));
+  FD_TRY(patch_io(h, h->latent_stage[slot], h->out_stage[slot]));
+  FD_CUDA(cudaGraphLaunch(h->exec, g));
+  FD_CUDA(cudaEventRecord(h->ev_graph[slot], g));
+  // the copy-out on the caller's stream: synchronising it covers this frame,
+  // while the next frame's graph can already run on host_stream
+  FD_CUDA(cudaStreamWaitEvent(s, h->ev_graph[slot], 0));
+  FD_CUDA(cudaMemcpyAsync(out_host, h->out_stage[slot], h->B * h->out_elems * h->io_elt,
                           cudaMemcpyDeviceToHost, s));
+  FD_CUDA(cudaEventRecord(h->ev_d2h[slot], s));
+  h->d2h_pending[slot] = true;
+  h->g_last = slot;
+  h->host_slot = slot ^ 1;
   h->last_stream = s;
   return FD_OK;
 }
@@ -1262,6 +1391,7 @@ const char* fd_error_string(fd_status_t s) {
     case FD_ERR_CUDA: return "CUDA error";
     case FD_ERR_TIMEOUT: return "device-side wait timed out";
     case FD_ERR_BAD_HANDLE: return "invalid handle";
+    case FD_ERR_BOUNDS: return "device-side bounds check failed (bounds-checked build)";
   }
   return "unknown status";
 }
@@ -1330,6 +1460,85 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
   return FD_OK;
 }
 
+fd_status_t fd_debug_read_ring(fd_handle* h, int block, int b, int slot, int kv, float* host_dst) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_read_ring: invalid handle");
+  const fd_config& c = h->cfg;
+  const bool refine = h->paper && block >= c.n_blocks;
+  const int n_all = c.n_blocks + (h->paper ? c.n_refine : 0);
+  const int slots = refine ? c.r_t * (c.window + 1) : c.window + 1;
+  if (block < 0 || block >= n_all || b < 0 || b >= h->B || slot < 0 || slot >= slots ||
+      (kv != 0 && kv != 1) || !host_dst)
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_read_ring: bad block/stream/slot/kv/dst");
+  FD_CUDA(cudaDeviceSynchronize());
+  const int G = c.n_kv_heads, Dh = c.head_dim, L = h->L;
+  const int layer = refine ? block - c.n_blocks : block;
+  const int rows = refine ? h->rkv_rows : h->kv_rows;
+  const int pitch = refine ? h->rvt_pitch : h->vt_pitch;
+  const char* kbase = static_cast<const char*>(refine ? h->rkc : h->kc);
+  const char* vbase = static_cast<const char*>(refine ? h->rvtc : h->vtc);
+  const size_t slab = (size_t(layer) * h->B + b) * G;      // first (layer, stream, group) slab
+  const size_t n = size_t(G) * L * Dh;
+  auto to_f32 = [&](const uint8_t* src, size_t i) {
+    return h->bf ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src)[i])
+                 : reinterpret_cast<const float*>(src)[i];
+  };
+  if (kv == 0) {
+    std::vector<uint8_t> raw(n * h->elt);
+    for (int g = 0; g < G; ++g) {
+      const size_t src = ((slab + g) * rows + size_t(slot) * L) * Dh * h->elt;
+      FD_CUDA(cudaMemcpy(raw.data() + size_t(g) * L * Dh * h->elt, kbase + src,
+                         size_t(L) * Dh * h->elt, cudaMemcpyDeviceToHost));
+    }
+    for (size_t i = 0; i < n; ++i) host_dst[i] = to_f32(raw.data(), i);
+  } else {
+    // V^T [G][Dh][pitch] -> [G][L][Dh]
+    std::vector<uint8_t> rowbuf(size_t(L) * h->elt);
+    for (int g = 0; g < G; ++g)
+      for (int d = 0; d < Dh; ++d) {
+        const size_t src = ((slab + g) * Dh + d) * pitch + size_t(slot) * L;
+        FD_CUDA(cudaMemcpy(rowbuf.data(), vbase + src * h->elt, size_t(L) * h->elt,
+                           cudaMemcpyDeviceToHost));
+        for (int n2 = 0; n2 < L; ++n2)
+          host_dst[(size_t(g) * L + n2) * Dh + d] = to_f32(rowbuf.data(), n2);
+      }
+  }
+  return FD_OK;
+}
+
+fd_status_t fd_debug_set_frame_index(fd_handle* h, int b, int64_t t, void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_set_frame_index: invalid handle");
+  if (b < 0 || b >= h->B || t < 0)
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_set_frame_index: bad stream or negative index");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
+  const long long v = t;
+  FD_CUDA(cudaMemcpyAsync(h->ctr + b, &v, 8, cudaMemcpyHostToDevice, s));
+  FD_CUDA(cudaStreamSynchronize(s));             // v lives on this stack frame
+  h->last_stream = s;
+  return FD_OK;
+}
+
+fd_status_t fd_debug_poison(fd_handle* h, int32_t what, void* stream) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_poison: invalid handle");
+  if (what & ~int32_t(FD_POISON_RING | FD_POISON_SPLIT_COUNTERS))
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_poison: unknown flags 0x%x", unsigned(what));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
+  if (what & FD_POISON_RING) {
+    // all-ones bytes: a NaN in both bf16 and fp32
+    FD_CUDA(cudaMemsetAsync(h->kc, 0xFF, h->k_bytes, s));
+    FD_CUDA(cudaMemsetAsync(h->vtc, 0xFF, h->v_bytes, s));
+    if (h->paper) {
+      FD_CUDA(cudaMemsetAsync(h->rkc, 0xFF, h->rk_bytes, s));
+      FD_CUDA(cudaMemsetAsync(h->rvtc, 0xFF, h->rv_bytes, s));
+    }
+  }
+  if ((what & FD_POISON_SPLIT_COUNTERS) && h->split_ctr)
+    FD_CUDA(cudaMemsetAsync(h->split_ctr, 0x7F, h->split_units() * 4, s));
+  h->last_stream = s;
+  return FD_OK;
+}
+
 fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, float* out_host) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_block_mlp: invalid handle");
   const fd_config& c = h->cfg;
@@ -1344,6 +1553,7 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   // stream; no timing events, no calibration records
   cudaGraph_t saved_graph = h->graph;
   cudaGraphNode_t saved_last = h->last_node;
+  const bool saved_is_kernel = h->last_is_kernel;
   const size_t saved_kinds = h->kinds.size();
   const int saved_timing = h->cfg.kernel_timing;
   unsigned* saved_amax = h->amax;
@@ -1352,11 +1562,13 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   FD_CUDA(cudaGraphCreate(&g, 0));
   h->graph = g;
   h->last_node = nullptr;
+  h->last_is_kernel = false;
   h->cfg.kernel_timing = 0;
   h->amax = nullptr;
   fd_status_t st = h->add_post_attention(block, h->backbone_io(0));
   h->graph = saved_graph;
   h->last_node = saved_last;
+  h->last_is_kernel = saved_is_kernel;
   h->kinds.resize(saved_kinds);
   h->cfg.kernel_timing = saved_timing;
   h->amax = saved_amax;
@@ -1378,10 +1590,16 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
 }  // extern "C"
 
 // Fixed device scratch of fd_decode_frame_static_scratch: the attention
-// key-splitting partials and counters of one frame, for handles whose need fits
-// (modest configurations). Zero at module load; every launch leaves its
-// counters at zero again.
+// key-splitting counters and partials of one frame, for handles whose need
+// fits (modest configurations). Layout, the same for every handle:
+//   [0, kStaticCtrBytes)            split counters, one int per unit, cleared
+//                                   by every call before its frame runs
+//   [kStaticCtrBytes, ...)          partial O, then partial (max, sum)
+// The counters never share bytes with another handle's partials, and the
+// clearing makes each call independent of what an earlier call (or one that
+// gave up on a timeout) left behind.
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+constexpr size_t kStaticCtrBytes = size_t(64) << 10;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 namespace {
@@ -1399,13 +1617,17 @@ fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent, voi
   const size_t units = h->split_units();
   const size_t o_bytes = units * h->n_split * 128 * 64 * 4;
   const size_t ml_bytes = units * h->n_split * 128 * 2 * 4;
-  const size_t need = round_up(o_bytes, 256) + round_up(ml_bytes, 256) + units * 4;
-  if (need > kStaticScratchBytes)
+  const size_t need = kStaticCtrBytes + round_up(o_bytes, 256) + ml_bytes;
+  if (units * 4 > kStaticCtrBytes || need > kStaticScratchBytes)
     return fail(FD_ERR_UNSUPPORTED,
                 "fd_decode_frame_static_scratch: attention scratch of %zu bytes exceeds the fixed %zu",
                 need, kStaticScratchBytes);
   int dev = 0;
   FD_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device)
+    return fail(FD_ERR_INVALID_ARG,
+                "fd_decode_frame_static_scratch: current device %d is not the handle's device %d",
+                dev, h->device);
   if (dev < 0 || dev >= 64) return fail(FD_ERR_UNSUPPORTED, "fd_decode_frame_static_scratch: device %d", dev);
   char* base = nullptr;
   {
@@ -1419,9 +1641,9 @@ fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent, voi
     for (AttnNode& an : h->attn_nodes) {
       TcAttnParams ap = an.p;
       if (fixed) {
-        ap.part_o = reinterpret_cast<float*>(base);
-        ap.part_ml = reinterpret_cast<float*>(base + round_up(o_bytes, 256));
-        ap.counter = reinterpret_cast<int*>(base + round_up(o_bytes, 256) + round_up(ml_bytes, 256));
+        ap.counter = reinterpret_cast<int*>(base);
+        ap.part_o = reinterpret_cast<float*>(base + kStaticCtrBytes);
+        ap.part_ml = reinterpret_cast<float*>(base + kStaticCtrBytes + round_up(o_bytes, 256));
       }
       CUtensorMap a = an.tmQ, b = an.tmK, c = an.tmV;
       void* args[] = {&a, &b, &c, &ap};
@@ -1435,10 +1657,24 @@ fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent, voi
     }
     return FD_OK;
   };
-  FD_TRY(set(true));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_TRY(join_user_stream(h, s));
+  FD_CUDA(cudaMemsetAsync(base, 0, units * 4, s));
+  const fd_status_t st_set = set(true);
+  if (st_set != FD_OK) {
+    const std::string msg = g_last_error;
+    set(false);                        // never leave the graph on the shared array
+    g_last_error = msg;
+    return st_set;
+  }
   const fd_status_t st = fd_decode_frame(h, latent, out, stream);
+  const std::string msg = g_last_error;
   const fd_status_t back = set(false);
-  return st != FD_OK ? st : back;
+  if (st != FD_OK) {
+    g_last_error = msg;
+    return st;
+  }
+  return back;
 }
 
 fd_status_t fd_mlp_fp8_scales(fd_handle* h, float* scales_out, int32_t cap, int32_t* n_out) {

@@ -54,6 +54,9 @@ struct TcAttnParams {
   float* part_o;      // [unit][n_split][128][64] unnormalised O
   float* part_ml;     // [unit][n_split][128][2] running max (log2 domain), sum
   int* counter;       // [unit] CTAs of the unit done so far (0 between launches)
+  // bounds of the bounds-checked build (FD_IN_BOUNDS)
+  int kv_rows;        // rows of one (layer, stream, group) slab of the ring
+  int n_slabs;        // slabs in the ring's tensor maps: layers x B x G
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -163,11 +166,6 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
   const int bs = blockIdx.z / p.n_split, split = blockIdx.z - bs * p.n_split;
   const int g = h / (p.H / p.G);
   const int lg = (p.layer * p.B + bs) * p.G + g;
-  const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
-  const int n_kt_all = (n_keys + 63) / 64;
-  // this CTA's key tiles: [j0, j0 + n_kt) (all of them without splitting)
-  const int j0 = split * n_kt_all / p.n_split;
-  const int n_kt = (split + 1) * n_kt_all / p.n_split - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -185,6 +183,14 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();                                 // Q, K, V and the frame state
+  griddep_launch();
+  int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
+  if (!FD_IN_BOUNDS(n_keys <= p.kv_rows && lg < p.n_slabs, p.status)) n_keys = 0;
+  const int n_kt_all = (n_keys + 63) / 64;
+  // this CTA's key tiles: [j0, j0 + n_kt) (all of them without splitting)
+  const int j0 = split * n_kt_all / p.n_split;
+  const int n_kt = (split + 1) * n_kt_all / p.n_split - j0;
 
   if (warp == 0) {
     if (lane == 0) {                                       // ---- TMA producer
@@ -258,6 +264,18 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
       if (valid < 64) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] = (c < valid) ? x[c] : -INFINITY;
+        // P is 0 for those keys, and their V^T columns (a ring slot not yet
+        // written since the reset, or the row padding) may hold anything: a
+        // NaN there would still reach O as 0 x NaN, so zero them in the
+        // stage before the PV product reads it. The stage's TMA load is
+        // complete (its barrier phase cannot move on before P(j) arrives).
+        const int st = j % ST;
+        if (!mbar_wait_warp(&kv_full[st], (j / ST) & 1, abort_flag, p.status)) { ok = false; break; }
+        uint8_t* vt = smem + S::kKV + st * S::kKVStage + 8192;   // [64 dims][128 B], 128-B swizzle
+        const int t = threadIdx.x - 64, d = t >> 1;
+        for (int c = valid + (t & 1); c < 64; c += 2)
+          *reinterpret_cast<uint16_t*>(vt + d * 128 + (((c >> 3) ^ (d & 7)) << 4) + (c & 7) * 2) = 0;
+        fence_proxy_async_smem();
       }
       float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
 #pragma unroll
@@ -319,7 +337,7 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
         store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
                                 size_t(h) * 64, v);
       }
-    } else {
+    } else if (FD_IN_BOUNDS(bs < p.B && split < p.n_split, p.status)) {   // uniform per CTA
       // this key range's partial result
       const size_t unit = (size_t(bs) * p.H + h) * gridDim.x + blockIdx.x;
       const size_t prow = (unit * p.n_split + split) * 128 + r;

@@ -71,4 +71,19 @@ __device__ __forceinline__ void report_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Bounds checks of the bounds-checked build (-DFD_DEBUG, libflashdec_debug.so):
+// every computed ring row, slot, V^T column, split-partial index and pixel
+// offset is tested before the access; a failed test records FD_ERR_BOUNDS in
+// the device status word and the access is skipped (no trap, the kernel runs
+// on). In the normal build FD_IN_BOUNDS is the constant true and costs nothing.
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+  if (!ok) report_status(status, FD_ERR_BOUNDS);
+  return ok;
+}
+#ifdef FD_DEBUG
+#define FD_IN_BOUNDS(cond, status) (::fd::in_bounds((cond), (status)))
+#else
+#define FD_IN_BOUNDS(cond, status) true
+#endif
+
 }  // namespace fd

@@ -13,11 +13,12 @@
 //   UP     bias -> temporal upsampling (Sec. 3.4, Eq. 3): output channels
 //          [tau D, (tau+1) D) become the residual stream of sub-frame tau
 //          (fp32 copy, storage-type copy, per-32-column sums of squares)
-// FP8 MLP (Sec. 4.6, static per-tensor scales):
-//   RESID_Q  as RESID, but the copy of x is FP8 E4M3, x / s_x (the MLP-up's
-//            A operand), instead of the storage type
-//   GELU_Q   dequantize (acc s_x s_w1) + RMSNorm row scale + bias + GELU ->
-//            FP8 hidden h / s_h (the MLP-down's A operand)
+// FP8 MLP (Sec. 4.6, static per-tensor scales; the MLP-up's FP8 input
+// e4m3(RMSNorm(x) / s_a) is written by mlp_norm_quant_kernel in between):
+//   RESID_Q  as RESID, without the storage-type copy of x (the MLP-up reads
+//            the FP8 input instead)
+//   GELU_Q   dequantize (acc s_a s_w1) + bias + GELU -> FP8 hidden h / s_h
+//            (the MLP-down's A operand)
 //   RESID with acc_scale = s_h s_w2 dequantizes the MLP-down product
 // Calibration (unquantized path): RESID and GELU can record max |value| of
 // their outputs into a device word (float bits, atomicMax).
@@ -40,7 +41,7 @@ enum EpiKind {
 // Kinds whose A operand is an RMSNorm input (their rows get the row scale);
 // a null EpiParams::ssq turns the scale off (the spatial MLP's second layer).
 constexpr bool epi_normed(int kind) {
-  return kind == EPI_QKV || kind == EPI_GELU || kind == EPI_FINAL || kind == EPI_GELU_Q;
+  return kind == EPI_QKV || kind == EPI_GELU || kind == EPI_FINAL;
 }
 
 struct EpiParams {
@@ -86,9 +87,12 @@ struct EpiParams {
   // FP8 MLP
   float acc_scale;       // dequantization of the accumulator (1: none)
   float q_inv;           // 1 / static scale of the FP8 output
-  void* x8;              // RESID_Q: [M][D] E4M3 copy of x
   // calibration: max |output| as float bits (null: off)
   unsigned* amax;
+  // bounds of the bounds-checked build (FD_IN_BOUNDS)
+  int* status;           // device status word
+  int n_sub;             // UP: sub-frames r_t of x32 / xb / ssq_out
+  int out_frames;        // FINAL: pixel frames per stream (C r_t)
 };
 
 // 64 floats * q_inv -> 64 E4M3 bytes (round to nearest even, saturating at
@@ -221,6 +225,9 @@ __device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int c
     const int dy = (col / P) % P;
     const size_t off = size_t(b) * p.out_stride + size_t(ct) * plane +
                        (size_t(i) * P + dy) * out_w + size_t(j) * P;
+    if (!FD_IN_BOUNDS(ct < p.out_frames && i < p.tok_h && off + P <= size_t(b + 1) * p.out_stride,
+                      p.status))
+      continue;
     if (p.out_bf16) store_vec<bf16, P>(static_cast<bf16*>(p.out) + off, acc + s);
     else store_vec<float, P>(static_cast<float*>(p.out) + off, acc + s);
   }
@@ -248,12 +255,16 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
         if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
         rope_head<DH>(v, n, fs, p);
         const int key = fs->slot * p.L + n;
+        if (!FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && b * p.L < p.M, p.status)) continue;
         T* dst = static_cast<T*>(p.kc) + ((size_t(b) * p.G + g) * p.kv_rows + key) * DH;
         store_vec<T, DH>(dst, v);
       } else {                                            // value group
         const int g = head - p.H - p.G;
         if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
         const int key = fs->slot * p.L + n;
+        if (!FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && key < p.vt_pitch && g < p.G &&
+                          b * p.L < p.M, p.status))
+          continue;
         T* dst = static_cast<T*>(p.vtc) + (size_t(b) * p.G + g) * DH * p.vt_pitch + key;
 #pragma unroll
         for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch] = from_f<T>(v[d]);
@@ -273,9 +284,7 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
       *reinterpret_cast<float4*>(x + c) = o;
       acc[c + 0] = o.x; acc[c + 1] = o.y; acc[c + 2] = o.z; acc[c + 3] = o.w;
     }
-    if constexpr (KIND == EPI_RESID_Q)
-      store_e4m3_64(static_cast<uint8_t*>(p.x8) + size_t(row) * p.D + col0, acc, p.q_inv);
-    else
+    if constexpr (KIND == EPI_RESID)
       store_vec<T, 64>(static_cast<T*>(p.xb) + size_t(row) * p.D + col0, acc);
     if (p.amax) record_amax(p.amax, acc);
     const int parts = p.D / 32;
@@ -293,14 +302,14 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
     store_vec<T, 64>(static_cast<T*>(p.hout) + size_t(row) * p.N + col0, acc);
     if (p.amax) record_amax(p.amax, acc);
   } else if constexpr (KIND == EPI_GELU_Q) {
-    const float sc = rs * p.acc_scale;
-    scale_bias<64>(acc, sc, p.bias, col0);
+    scale_bias<64>(acc, p.acc_scale, p.bias, col0);
 #pragma unroll
     for (int c = 0; c < 64; ++c) acc[c] = gelu_erf(acc[c]);
     store_e4m3_64(static_cast<uint8_t*>(p.hout) + size_t(row) * p.N + col0, acc, p.q_inv);
   } else if constexpr (KIND == EPI_UP) {
     const int tau = col0 / p.D, c0 = col0 - tau * p.D;
     const size_t r = size_t(tau) * p.M + row;             // row of sub-frame tau
+    if (!FD_IN_BOUNDS(tau < p.n_sub, p.status)) return;
     scale_bias<64>(acc, 1.f, p.bias, col0);
     float* x = p.x32 + r * p.D + c0;
 #pragma unroll

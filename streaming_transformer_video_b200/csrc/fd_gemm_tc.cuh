@@ -83,6 +83,8 @@ __global__ void __launch_bounds__(gemm_threads(KIND), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();                                     // inputs of the previous kernel
+  griddep_launch();
 
   if (warp == 0) {
     if (lane == 0) {                                  // ---- TMA producer

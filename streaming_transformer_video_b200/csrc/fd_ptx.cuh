@@ -22,6 +22,22 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch: the frame graph links consecutive kernels
+// with programmatic edges, so a kernel's prologue (barrier set-up, TMEM
+// allocation, tensor-map prefetch) overlaps the tail of the kernel before it.
+// Every kernel calls griddep_wait() in every thread before its first access
+// to global memory that another kernel of the frame writes or reads; it
+// returns once the preceding grid has completed and its writes are visible.
+// griddep_launch() allows the next kernel to begin launching. Both are no-ops
+// for a launch without a programmatic dependency.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -14,39 +14,40 @@
 namespace fd {
 
 // ---------------------------------------------------------------- step_begin
-// Frame state of one streamed frame with absolute index t in a ring of `cap`
-// slots: slot = t mod cap; n_valid = min(t, cap - 1) + 1; temporal RoPE
-// angles t * theta^(-2m/d_t) reduced mod 2 pi in fp64 so they stay exact for
-// any stream length.
-__device__ void frame_state(FrameState* fs, long long t, int cap, int head_dim, float theta) {
-  fs->t = t;
-  fs->slot = int(t % cap);
-  fs->n_valid = int(t < cap - 1 ? t : cap - 1) + 1;
-  const int dt = head_dim / 4;
-  const double two_pi = 6.283185307179586476925286766559;
-  for (int m = 0; m < dt / 2; ++m) {
-    const double freq = pow(double(theta), -2.0 * m / dt);
-    const double ang = fmod(double(t) * freq, two_pi);
-    fs->rope_t[m] = make_float2(float(cos(ang)), float(sin(ang)));
-  }
-}
-
 // B video streams, each with its own counter ctr[b] and 1 + n_sub states
 // fs[b (1 + n_sub) + k]:
 //   k = 0: latent frame t = ctr[b] in the backbone ring of W+1 frames;
 //   k = 1 + tau, tau < n_sub (paper head, n_sub = r_t): sub-frame t r_t + tau
 //   in the refinement ring of r_t (W+1) sub-frames (paper Sec. 3.4, Step 2).
-// Every counter then advances by one. One CTA of 32 threads.
-__global__ void step_begin_kernel(long long* ctr, FrameState* fs, int W, int head_dim,
-                                  float theta, int n_sub, int B) {
+// A frame with absolute index t in a ring of `cap` slots gets slot =
+// t mod cap, n_valid = min(t, cap - 1) + 1, and temporal RoPE angles
+// t * theta^(-2m/d_t) (inv_freq[m], fp64 from the host) reduced mod 2 pi in
+// fp64, so they stay exact for any stream length. One thread per (state,
+// angle); every counter then advances by one. One CTA.
+__global__ void __launch_bounds__(256) step_begin_kernel(long long* ctr, FrameState* fs, int W,
+                                                         int n_pairs, const double* inv_freq,
+                                                         int n_sub, int B) {
   __shared__ long long t0[kMaxStreams];
+  griddep_wait();
+  griddep_launch();
   for (int b = threadIdx.x; b < B; b += blockDim.x) t0[b] = ctr[b];
   __syncthreads();
   const int per = 1 + n_sub;
-  for (int i = threadIdx.x; i < B * per; i += blockDim.x) {
-    const int b = i / per, k = i - b * per;
-    if (k == 0) frame_state(fs + i, t0[b], W + 1, head_dim, theta);
-    else frame_state(fs + i, t0[b] * n_sub + (k - 1), n_sub * (W + 1), head_dim, theta);
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = threadIdx.x; i < B * per * n_pairs; i += blockDim.x) {
+    const int st = i / n_pairs, m = i - st * n_pairs;
+    const int b = st / per, k = st - b * per;
+    const long long t = k == 0 ? t0[b] : t0[b] * n_sub + (k - 1);
+    const int cap = k == 0 ? W + 1 : n_sub * (W + 1);
+    FrameState* f = fs + st;
+    if (m == 0) {
+      f->t = t;
+      f->slot = int(t % cap);
+      f->n_valid = int(t < cap - 1 ? t : cap - 1) + 1;
+    }
+    double sn, cs;
+    sincos(fmod(double(t) * inv_freq[m], two_pi), &sn, &cs);
+    f->rope_t[m] = make_float2(float(cs), float(sn));
   }
   __syncthreads();
   for (int b = threadIdx.x; b < B; b += blockDim.x) ctr[b] = t0[b] + 1;
@@ -82,6 +83,7 @@ struct EmbedParams {
   float* x32;             // [M][D]
   void* xb;               // [M][D] storage type
   float* ssq;             // [M][D/32]
+  int* status;            // device status word (bounds-checked build)
 };
 
 constexpr int kEmbedTok = 8;
@@ -92,6 +94,8 @@ constexpr int kEmbedTok = 8;
 template <typename T>
 __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
   extern __shared__ float u[];                          // [kEmbedTok][c_in]
+  griddep_wait();
+  griddep_launch();
   const int n0 = blockIdx.x * kEmbedTok;
   for (int idx = threadIdx.x; idx < kEmbedTok * p.c_in; idx += blockDim.x) {
     const int tk = idx / p.c_in, ch = idx - tk * p.c_in;
@@ -102,7 +106,8 @@ __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
       const int c = ch / (p.p * p.p), dy = (ch / p.p) % p.p, dx = ch % p.p;
       const int i = nt / p.tok_w, j = nt - (nt / p.tok_w) * p.tok_w;
       const size_t off = ((size_t(b) * p.C + c) * p.Hl + i * p.p + dy) * p.Wl + j * p.p + dx;
-      v = p.latent_bf16 ? __bfloat162float(static_cast<const bf16*>(p.latent)[off])
+      if (FD_IN_BOUNDS(i * p.p + dy < p.Hl && j * p.p + dx < p.Wl, p.status))
+        v = p.latent_bf16 ? __bfloat162float(static_cast<const bf16*>(p.latent)[off])
                         : static_cast<const float*>(p.latent)[off];
     }
     u[idx] = v;
@@ -134,6 +139,61 @@ __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
   }
 }
 
+// ---------------------------------------------------------------- MLP input (FP8)
+// FP8 MLP (paper Sec. 4.6, static-calibrated FP8 quantization of the MLP
+// layers): the first MLP Linear multiplies the FP8 image of its own input,
+// the RMSNorm output a = x r g (r = 1/sqrt(mean(x^2) + eps), gain g), with
+// the static scale s_a: x8 = e4m3(a / s_a), round to nearest even,
+// saturating. With amax set (calibration of the unquantized path) the kernel
+// records max |a| instead and writes nothing. r comes from the per-32-column
+// sums of squares the producer of x emitted. One warp per row; D a multiple
+// of 128. Bound by memory (x read once, one byte written per element).
+struct NormQuantParams {
+  const float* x32;       // [M][D] residual stream
+  const float* ssq;       // [M][D/32] sums of squares of x32
+  const float* g;         // [D] RMSNorm gain
+  uint8_t* x8;            // [M][D] E4M3 codes of a / s_a (null with amax)
+  unsigned* amax;         // calibration: max |a| as float bits (null: quantize)
+  int M, D;
+  float inv_d, eps;
+  float q_inv;            // 1 / s_a
+};
+
+__global__ void __launch_bounds__(256) mlp_norm_quant_kernel(NormQuantParams p) {
+  griddep_wait();
+  griddep_launch();
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= p.M) return;
+  const int parts = p.D / 32;
+  float s = 0.f;
+  for (int i = lane; i < parts; i += 32) s += p.ssq[size_t(row) * parts + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float r = rsqrtf(s * p.inv_d + p.eps);
+  const float4* x = reinterpret_cast<const float4*>(p.x32 + size_t(row) * p.D);
+  const float4* g = reinterpret_cast<const float4*>(p.g);
+  float m = 0.f;
+  for (int c = lane; c < p.D / 4; c += 32) {
+    const float4 v = x[c], gg = __ldg(g + c);
+    const float a0 = v.x * r * gg.x, a1 = v.y * r * gg.y, a2 = v.z * r * gg.z, a3 = v.w * r * gg.w;
+    if (p.amax) {
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(a2), fabsf(a3))));
+    } else {
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(a0 * p.q_inv, a1 * p.q_inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(a2 * p.q_inv, a3 * p.q_inv), __NV_SATFINITE, __NV_E4M3);
+      reinterpret_cast<uint32_t*>(p.x8 + size_t(row) * p.D)[c] = uint32_t(lo) | (uint32_t(hi) << 16);
+    }
+  }
+  if (p.amax) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) atomicMax(p.amax, __float_as_uint(m));   // non-negative floats order as their bits
+  }
+}
+
 // ---------------------------------------------------------------- simt_gemm
 // C[M][N] = A[M][K] * B[N][K]^T, fp32, one thread per row and 64 columns,
 // then the fused epilogue. CTA = 128 rows x 64 columns; K in chunks of 32.
@@ -141,6 +201,8 @@ template <int KIND, int DH>
 __global__ void __launch_bounds__(128) simt_gemm_kernel(const float* A, const float* B, int K,
                                                         EpiParams p) {
   __shared__ float Bs[64][33];
+  griddep_wait();
+  griddep_launch();
   const int row = blockIdx.x * 128 + threadIdx.x;
   const int col0 = blockIdx.y * 64;
   float acc[64];
@@ -185,11 +247,14 @@ struct AttnParams {
 // online softmax in base 2. Keys [0, n_valid*L) are the valid ring slots.
 template <int DH>
 __global__ void __launch_bounds__(64) simt_attn_kernel(AttnParams p) {
+  griddep_wait();
+  griddep_launch();
   __shared__ float Ks[32][DH + 1];
   __shared__ float Vs[32][DH + 1];
   const int h = blockIdx.y, g = h / (p.H / p.G), bs = blockIdx.z;
   const int row = blockIdx.x * 64 + threadIdx.x;
-  const int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
+  int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
+  if (!FD_IN_BOUNDS(n_keys <= p.kv_rows, p.status)) n_keys = 0;
   const float* qp = static_cast<const float*>(p.q) +
                     ((size_t(h) * p.B + bs) * p.L + (row < p.L ? row : 0)) * DH;
   float q[DH], o[DH];

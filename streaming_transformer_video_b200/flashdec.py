@@ -15,20 +15,26 @@ from typing import Dict, List, Optional, Tuple
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libflashdec.so")
+# FLASHDEC_LIB=debug selects the bounds-checked build (libflashdec_debug.so,
+# same ABI; out-of-range device accesses are skipped and reported as
+# FD_ERR_BOUNDS by fd_status)
+LIB_PATH = os.path.join(_HERE, "libflashdec_debug.so" if os.environ.get("FLASHDEC_LIB") == "debug"
+                        else "libflashdec.so")
 
 FD_OK, FD_ERR_INVALID_ARG, FD_ERR_UNSUPPORTED, FD_ERR_OOM = 0, -1, -2, -3
-FD_ERR_CUDA, FD_ERR_TIMEOUT, FD_ERR_BAD_HANDLE = -4, -5, -6
+FD_ERR_CUDA, FD_ERR_TIMEOUT, FD_ERR_BAD_HANDLE, FD_ERR_BOUNDS = -4, -5, -6, -7
+FD_POISON_RING, FD_POISON_SPLIT_COUNTERS = 1, 2
 FD_F32, FD_BF16 = 0, 1
 KERNEL_KINDS = ["step_begin", "embed", "qkv", "attn", "oproj", "mlp_up", "mlp_down", "final",
-                "upsample", "spatial"]
+                "upsample", "spatial", "mlp_norm"]
 HEAD_MODES = {"linear": 0, "paper": 1}
 
 EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "fd_destroy",
            "fd_status", "fd_error_string", "fd_last_error", "fd_frame_index", "fd_device_bytes",
            "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
            "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp",
-           "fd_reset_stream", "fd_stream_frame_index", "fd_decode_frame_static_scratch"]
+           "fd_reset_stream", "fd_stream_frame_index", "fd_decode_frame_static_scratch",
+           "fd_debug_read_ring", "fd_debug_poison", "fd_debug_set_frame_index"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -60,7 +66,7 @@ class FDWeightsC(ctypes.Structure):
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"libflashdec.so not found at {path}; build it with "
+        raise ImportError(f"{os.path.basename(path)} not found at {path}; build it with "
                           "`python -m streaming_transformer_video_b200.csrc.build`")
     lib = ctypes.CDLL(path)
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -88,6 +94,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_reset_stream.argtypes = [vp, i32, vp]
     lib.fd_decode_frame_static_scratch.argtypes = [vp, vp, vp, vp]
     lib.fd_stream_frame_index.argtypes = [vp, i32, ctypes.POINTER(i64)]
+    lib.fd_debug_read_ring.argtypes = [vp, i32, i32, i32, i32, _PF]
+    lib.fd_debug_poison.argtypes = [vp, i32, vp]
+    lib.fd_debug_set_frame_index.argtypes = [vp, i32, i64, vp]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
             getattr(lib, name).restype = i32
@@ -172,7 +181,7 @@ class FlashDecoder:
     "b{l}.w1", "b{l}.b1", "b{l}.w2", "b{l}.b2", "final_g", "out_w", "out_b".
     With cfg.head == "paper" also "up_w", "up_b", "sp1_w", "sp1_b" and the
     refinement blocks "r{l}.*" (same keys as "b{l}.*"), l < cfg.n_refine.
-    With cfg.mlp_fp8 also the static FP8 scales "b{l}.fp8_sx", "b{l}.fp8_sh"
+    With cfg.mlp_fp8 also the static FP8 scales "b{l}.fp8_sa", "b{l}.fp8_sh"
     (and "r{l}.*") of every block, e.g. from mlp_fp8_scales() of a handle
     created with record_mlp_amax=True.
     """
@@ -211,7 +220,7 @@ class FlashDecoder:
         if self.c.mlp_fp8:
             pairs = []
             for p in prefixes:
-                a = np.array([weights[p + "fp8_sx"], weights[p + "fp8_sh"]], dtype=np.float32)
+                a = np.array([weights[p + "fp8_sa"], weights[p + "fp8_sh"]], dtype=np.float32)
                 keep.append(a)
                 pairs.append(a.ctypes.data_as(_PF))
             arr = (_PF * len(pairs))(*pairs)
@@ -304,6 +313,27 @@ class FlashDecoder:
                "fd_debug_read_slot")
         return out
 
+    def read_ring(self, block: int, b: int, slot: int, kv: int) -> np.ndarray:
+        """Ring slot of any block (refinement blocks follow the backbone's) and
+        stream b, as float32 [G][L_frm][D_h] (kv 0 = keys, 1 = values)."""
+        cfg = self.cfg
+        L = (cfg.grid_h // cfg.patch) * (cfg.grid_w // cfg.patch)
+        out = np.empty((cfg.n_kv_heads, L, cfg.head_dim), dtype=np.float32)
+        _check(self._lib.fd_debug_read_ring(self.h, block, b, slot, kv, out.ctypes.data_as(_PF)),
+               "fd_debug_read_ring")
+        return out
+
+    def debug_poison(self, what: int, stream=None):
+        """Fill the ring caches with NaN (FD_POISON_RING) and/or the split
+        counters with garbage (FD_POISON_SPLIT_COUNTERS)."""
+        _check(self._lib.fd_debug_poison(self.h, int(what), _stream_handle(stream)),
+               "fd_debug_poison")
+
+    def debug_set_frame_index(self, t: int, b: int = 0, stream=None):
+        """Treat the next frame of stream b as frame t (tests of long videos)."""
+        _check(self._lib.fd_debug_set_frame_index(self.h, int(b), int(t), _stream_handle(stream)),
+               "fd_debug_set_frame_index")
+
     def debug_block_mlp(self, block: int, x: np.ndarray) -> np.ndarray:
         """x + b_o + MLP(x + b_o) of block `block` for a residual stream x
         [L_frm][D] (float32), through the block's own kernels."""
@@ -314,7 +344,7 @@ class FlashDecoder:
         return out
 
     def mlp_fp8_scales(self) -> Dict[str, float]:
-        """Static FP8 scales {"b{l}.fp8_sx": .., "b{l}.fp8_sh": .., ...} from
+        """Static FP8 scales {"b{l}.fp8_sa": .., "b{l}.fp8_sh": .., ...} from
         the MLP ranges recorded since the last reset (record_mlp_amax=True)."""
         n = ctypes.c_int32()
         _check(self._lib.fd_mlp_fp8_scales(self.h, None, 0, ctypes.byref(n)), "fd_mlp_fp8_scales")
@@ -323,7 +353,7 @@ class FlashDecoder:
                "fd_mlp_fp8_scales")
         res = {}
         for i, p in enumerate(self._prefixes):
-            res[p + "fp8_sx"], res[p + "fp8_sh"] = float(out[2 * i]), float(out[2 * i + 1])
+            res[p + "fp8_sa"], res[p + "fp8_sh"] = float(out[2 * i]), float(out[2 * i + 1])
         return res
 
     def kernel_ms(self) -> List[Tuple[str, float]]:

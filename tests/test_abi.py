@@ -58,7 +58,7 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
 
 def test_error_strings():
     lib = fdb.lib()
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         s = lib.fd_error_string(code).decode()
         assert s and s != "unknown status"
     assert lib.fd_error_string(-99).decode() == "unknown status"
@@ -150,6 +150,10 @@ def test_bad_handle_calls():
     assert lib.fd_debug_block_mlp(None, 0, None, None) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_reset_stream(None, 0, None) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_stream_frame_index(None, 0, ctypes.byref(t)) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_decode_frame_static_scratch(None, None, None, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_read_ring(None, 0, 0, 0, 0, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_poison(None, fdb.FD_POISON_RING, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_set_frame_index(None, 0, 5, None) == fdb.FD_ERR_BAD_HANDLE
     # a pointer to memory that is not a handle (magic check)
     junk = (ctypes.c_uint32 * 64)()
     assert lib.fd_reset(ctypes.cast(junk, ctypes.c_void_p), None) == fdb.FD_ERR_BAD_HANDLE

@@ -79,9 +79,9 @@ def test_small_bf16_fp8_mlp_matches_oracle(kw):
 @pytest.mark.parametrize("fp8", [1, 0])
 @pytest.mark.parametrize("kw", [dict(), dict(head="paper", n_refine=2, window=1)])
 def test_block_mlp_on_identical_inputs(fp8, kw):
-    # Both sides get the same float32 residual stream, so the E4M3 codes of
-    # x + b_o are identical and only the hidden activation's rounding can
-    # differ, where its float32 value lies within ~1e-6 of an E4M3 boundary.
+    # Both sides get the same float32 residual stream x + b_o; the E4M3 codes
+    # of its RMSNorm output and of the hidden activation can differ only
+    # where a float32 value lies within ~1e-6 of an E4M3 rounding boundary.
     from streaming_transformer_video_b200 import FlashDecoder
     from oracle import flashdec_oracle as fo
     cfg = small_bf16(frames=3, **kw)
@@ -97,9 +97,9 @@ def test_block_mlp_on_identical_inputs(fp8, kw):
         prefixes += [f"r{l}." for l in range(cfg.n_refine)]
     try:
         for i, p in enumerate(prefixes):
-            # a stream in the calibrated range (max |x| about 448 s_x)
-            x = (rng.standard_normal((cfg.L_frm, cfg.d_model)) * 100 * scales[p + "fp8_sx"])
-            x = x.astype(np.float32)
+            # a residual stream of the decoder's magnitude; its RMSNorm output
+            # lies in the calibrated range whatever the scale of x
+            x = (rng.standard_normal((cfg.L_frm, cfg.d_model)) * 3.0).astype(np.float32)
             got = dec.debug_block_mlp(i, x).astype(np.float64)
             xp = (x.astype(np.float64) + w64[p + "bo"]).astype(np.float32).astype(np.float64)
             ref = fo.mlp(cfg8, w64, p, xp)
