@@ -152,13 +152,19 @@ class ClockSampler:
         rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4)
                           if r[5 + i].strip().lower() == "active"})
         load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
         return {"sm_mhz": float(np.median(load)) if load else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows),
+                # SM clock range and power under load: per-step latency drift
+                # over the timed region follows the clock when the power cap acts
+                "sm_mhz_range": [min(load), max(load)] if load else None,
+                "power_w_max": max(pw) if pw else None,
+                "sm_mhz_by_sample": [int(x) for x in load][:400]}
 
 
 # ------------------------------------------------------------------ dist
@@ -339,6 +345,7 @@ def run_flashdec(args):
     time.sleep(0.3)
     barrier(dist)
     torch.cuda.synchronize()
+    mem_before = torch.cuda.mem_get_info()[0]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -349,6 +356,7 @@ def run_flashdec(args):
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    mem_after = torch.cuda.mem_get_info()[0]
     # device time of every attention launch of the last timed frame (CUDA
     # events recorded inside the graph; each replay overwrites them, so only
     # the last frame's are readable without syncing between frames)
@@ -450,6 +458,9 @@ def run_flashdec(args):
         "clocks": clk,
         "gpu_launches": launches * args.steps,
         "device_bytes": dev_bytes,
+        # free device memory right before and after the timed steps: the
+        # decoder allocates nothing per frame, so the two are equal
+        "device_free_bytes_before_after": [int(mem_before), int(mem_after)],
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
     }
@@ -473,7 +484,7 @@ def run_flashdec(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=14)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="flashdec", choices=["flashdec", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(fd_synth.CONFIGS))

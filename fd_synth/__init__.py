@@ -126,6 +126,11 @@ CONFIGS: Dict[str, FDConfig] = {
     # (8160 tokens), 7 frames, 16 blocks.
     "1080p_wan22": FDConfig("1080p_wan22", 48, 68, 120, 1, 1024, 16, 16, 64,
                             16, 4, 2, 3, 4, 16, 1, "bf16", 7),
+    # the same 1080p decoder with W = 1 (the paper's deployed W_frm = 2: the
+    # current latent frame plus one previous frame, Sec. 4.4 "Window Size
+    # Ablation"), a context row beside the W = 2 workload
+    "1080p_wan22_w1": FDConfig("1080p_wan22_w1", 48, 68, 120, 1, 1024, 16, 16, 64,
+                               16, 4, 1, 3, 4, 16, 1, "bf16", 7),
     # long-stream Wan2.2-shaped 720p: 48ch, 45x80 grid, patch 1 (3600 tokens),
     # 200 frames, 16 blocks.
     "long720p_wan22": FDConfig("long720p_wan22", 48, 45, 80, 1, 1024, 16, 16,

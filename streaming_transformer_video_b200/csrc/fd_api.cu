@@ -434,7 +434,7 @@ bool valid_handle(const fd_handle* h) { return h && h->magic == kMagic; }
 template <int BN, int KIND, bool F8>
 fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
   constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  using S = TcGemmSmem<BN, STAGES>;
+  using S = TcGemmSmem<BN, STAGES, KIND>;
   const void* f = reinterpret_cast<const void*>(&tc_gemm_kernel<BN, STAGES, KIND, 64, F8>);
   FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc));
   const int tiles = ((M + 127) / 128) * (N / BN);
@@ -774,7 +774,7 @@ fd_status_t fd_handle::build_graph() {
     embed_p.status = status;
     const void* f = bf ? reinterpret_cast<const void*>(&embed_kernel<bf16>)
                        : reinterpret_cast<const void*>(&embed_kernel<float>);
-    embed_launch = KernelLaunch{f, dim3((M + kEmbedTok - 1) / kEmbedTok), dim3(256),
+    embed_launch = KernelLaunch{f, dim3((M + kEmbedTok - 1) / kEmbedTok), dim3(kEmbedThreads),
                                 size_t(kEmbedTok) * c_in * 4, FD_K_EMBED};
     void* args[] = {&embed_p};
     FD_TRY(add_kernel(embed_launch, args, &embed_node));

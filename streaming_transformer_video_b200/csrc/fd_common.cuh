@@ -60,6 +60,22 @@ __device__ __forceinline__ void store_row<bf16, 8>(bf16* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = u;
 }
 
+// Four consecutive values as T (one 16-byte or 8-byte store).
+template <typename T> __device__ __forceinline__ void store_quad(T* dst, const float* v);
+template <>
+__device__ __forceinline__ void store_quad<float>(float* dst, const float* v) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void store_quad<bf16>(bf16* dst, const float* v) {
+  __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 p1 = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&p0);
+  u.y = *reinterpret_cast<uint32_t*>(&p1);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
 template <typename T, int n>
 __device__ __forceinline__ void store_vec(T* dst, const float* v) {
 #pragma unroll

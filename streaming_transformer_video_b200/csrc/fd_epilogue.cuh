@@ -233,6 +233,149 @@ __device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int c
   }
 }
 
+// Residual epilogue (RESID, RESID_Q) for a whole warp: thread `lane` holds
+// columns col0 .. col0+63 of row row0 + lane. Done row by row, each thread
+// would touch its own 256-byte row of x, so every warp-wide access would span
+// 32 rows. Instead the accumulator goes through a [32][kResidPitch] fp32 tile
+// of shared memory, 32 columns at a time, and 8 lanes cover one row: every
+// load and store of x (fp32), its storage-type copy and the sums of squares
+// is then a run of 128 (or 64) contiguous bytes per row. Rows past M are
+// skipped; the warp stays converged for the shuffles.
+constexpr int kResidPitch = 36;          // floats per tile row (conflict-free float4)
+
+template <int KIND, typename T>
+__device__ __forceinline__ void resid_epilogue64(const EpiParams& p, int row0, int col0,
+                                                 const float* acc, float* tile, int lane) {
+  const int parts = p.D / 32;
+  const float sc = p.acc_scale;
+  const int c4 = lane & 7, sub = lane >> 3;
+  // all 16 of this lane's residual reads first (they do not depend on the
+  // accumulator), so that they are in flight together
+  float4 xin[2][8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int row = row0 + 4 * it + sub;
+      xin[h][it] = row < p.M ? *reinterpret_cast<const float4*>(p.x32 + size_t(row) * p.D + col0 +
+                                                               32 * h + 4 * c4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float4* mine = reinterpret_cast<float4*>(tile + lane * kResidPitch);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      mine[k] = make_float4(acc[32 * h + 4 * k], acc[32 * h + 4 * k + 1], acc[32 * h + 4 * k + 2],
+                            acc[32 * h + 4 * k + 3]);
+    __syncwarp();
+    const int col = col0 + 32 * h + 4 * c4;
+    const float4 bb = bias4(p.bias, col);
+    float m = 0.f;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = 4 * it + sub, row = row0 + rr;
+      const bool in = row < p.M;
+      const float4 a = reinterpret_cast<const float4*>(tile + rr * kResidPitch)[c4];
+      float4 o = xin[h][it];
+      o.x += a.x * sc + bb.x;
+      o.y += a.y * sc + bb.y;
+      o.z += a.z * sc + bb.z;
+      o.w += a.w * sc + bb.w;
+      if (in) {
+        *reinterpret_cast<float4*>(p.x32 + size_t(row) * p.D + col) = o;
+        if constexpr (KIND == EPI_RESID) {
+          const float v[4] = {o.x, o.y, o.z, o.w};
+          store_quad<T>(static_cast<T*>(p.xb) + size_t(row) * p.D + col, v);
+        }
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+      }
+      float ss = o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      if (in && c4 == 0) p.ssq_out[size_t(row) * parts + (col0 + 32 * h) / 32] = ss;
+    }
+    if (p.amax) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) atomicMax(p.amax, __float_as_uint(m));
+    }
+    __syncwarp();
+  }
+}
+
+// QKV epilogue for a whole warp (tcgen05 path, bf16, D_h = 64): thread `lane`
+// holds head col0 / 64 of token row0 + lane. The math is the per-thread QKV
+// epilogue's; the query and key rows (128 bytes per token) then go through a
+// [32][kQkvPitch] bf16 tile of shared memory so that 8 lanes store one token's
+// row: each warp-wide store covers 4 whole rows instead of touching 32. The
+// transposed value rows keep the per-thread stores (32 consecutive keys of
+// one dimension per warp-wide store are already contiguous). Rows past M do
+// the arithmetic on clamped indices and store nothing.
+constexpr int kQkvPitch = 72;            // bf16 per tile row (conflict-free 16-byte access)
+
+__device__ __forceinline__ void warp_store_rows64(bf16* dst, const float* v, bf16* tile, int lane) {
+  // this lane's row -> tile, then 4 rows per step, 16 bytes per lane
+  uint4* mine = reinterpret_cast<uint4*>(tile + lane * kQkvPitch);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * k + 2 * i], v[8 * k + 2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    mine[k] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __syncwarp();
+  const int c = lane & 7, sub = lane >> 3;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int rr = 4 * it + sub;
+    bf16* d = reinterpret_cast<bf16*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(dst), rr));
+    const uint4 u = reinterpret_cast<const uint4*>(tile + rr * kQkvPitch)[c];
+    if (d) reinterpret_cast<uint4*>(d)[c] = u;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void qkv_epilogue64(const EpiParams& p, int row, int col0, float* acc,
+                                               float rs, bf16* tile, int lane) {
+  constexpr int DH = 64;
+  const bool valid = row < p.M;
+  const int rowc = valid ? row : 0;
+  const int b = rowc / p.L, n = rowc - b * p.L;            // stream, token
+  const FrameState* fs = p.fs + size_t(b) * p.fs_stride;
+  float* v = acc;
+  const int head = col0 / DH;
+  scale_bias<DH>(v, rs, p.bias, col0);
+  bf16* dst = nullptr;
+  if (head < p.H) {                                        // query head (warp-uniform)
+    rope_head<DH>(v, n, fs, p);
+    if (valid) dst = static_cast<bf16*>(p.q) + (size_t(head) * p.M + row) * DH;
+    warp_store_rows64(dst, v, tile, lane);
+  } else if (head < p.H + p.G) {                           // key group
+    const int g = head - p.H;
+    if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
+    rope_head<DH>(v, n, fs, p);
+    const int key = fs->slot * p.L + n;
+    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && b * p.L < p.M, p.status))
+      dst = static_cast<bf16*>(p.kc) + ((size_t(b) * p.G + g) * p.kv_rows + key) * DH;
+    warp_store_rows64(dst, v, tile, lane);
+  } else {                                                 // value group
+    const int g = head - p.H - p.G;
+    if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
+    const int key = fs->slot * p.L + n;
+    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && key < p.vt_pitch && g < p.G &&
+                              b * p.L < p.M, p.status)) {
+      bf16* d = static_cast<bf16*>(p.vtc) + (size_t(b) * p.G + g) * DH * p.vt_pitch + key;
+#pragma unroll
+      for (int i = 0; i < DH; ++i) d[size_t(i) * p.vt_pitch] = __float2bfloat16_rn(v[i]);
+    }
+  }
+}
+
 // acc[64]: columns col0 .. col0+63 of token `row` (row < M guaranteed).
 template <int KIND, typename T, int DH>
 __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0, float* acc,

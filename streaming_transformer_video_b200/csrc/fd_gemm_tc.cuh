@@ -27,14 +27,23 @@
 
 namespace fd {
 
-template <int BN, int STAGES>
+__host__ __device__ constexpr bool epi_resid(int kind) {
+  return kind == EPI_RESID || kind == EPI_RESID_Q;
+}
+
+template <int BN, int STAGES, int KIND = EPI_QKV>
 struct TcGemmSmem {
   static constexpr int kATile = 128 * 64 * 2;        // bytes
   static constexpr int kBTile = BN * 64 * 2;
   static constexpr int kStage = kATile + kBTile;
   static constexpr int kBarOff = STAGES * kStage;
   // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], tmem slot, abort
-  static constexpr int kBytes = kBarOff + (2 * STAGES + 4) * 8 + 16;
+  static constexpr int kEpiOff = kBarOff + (2 * STAGES + 4) * 8 + 16;
+  // residual epilogues: per epilogue warp a [32 rows][36] fp32 transpose tile;
+  // QKV: per epilogue warp a [32 rows][72] bf16 tile
+  static constexpr int kEpiBytes = epi_resid(KIND) ? 4 * 32 * kResidPitch * 4
+                                   : KIND == EPI_QKV ? 4 * 32 * kQkvPitch * 2 : 0;
+  static constexpr int kBytes = kEpiOff + kEpiBytes;
   static constexpr int kAlloc = kBytes + 1024;        // slack for 1024-B alignment
 };
 
@@ -47,7 +56,7 @@ template <int BN, int STAGES, int KIND, int DH, bool F8 = false>
 __global__ void __launch_bounds__(gemm_threads(KIND), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int K, EpiParams ep, int* status) {
-  using S = TcGemmSmem<BN, STAGES>;
+  using S = TcGemmSmem<BN, STAGES, KIND>;
   constexpr int kEpiThreads = gemm_epi_threads(KIND);
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   constexpr uint32_t kTmemCols = 2 * BN;              // power of two: 128, 256 or 512
@@ -159,7 +168,16 @@ __global__ void __launch_bounds__(gemm_threads(KIND), 1)
         float acc[64];
 #pragma unroll
         for (int i = 0; i < 32; ++i) { acc[i] = __uint_as_float(r0[i]); acc[32 + i] = __uint_as_float(r1[i]); }
-        if (row < M) epilogue64<KIND, bf16, DH>(ep, row, n_blk * BN + c, acc, rs);
+        if constexpr (epi_resid(KIND)) {
+          // whole warp: rows m_blk*128 + 32*quarter .. +31 through a transpose tile
+          float* tile = reinterpret_cast<float*>(smem + S::kEpiOff) + quarter * 32 * kResidPitch;
+          resid_epilogue64<KIND, bf16>(ep, m_blk * 128 + quarter * 32, n_blk * BN + c, acc, tile, lane);
+        } else if constexpr (KIND == EPI_QKV) {
+          bf16* tile = reinterpret_cast<bf16*>(smem + S::kEpiOff) + quarter * 32 * kQkvPitch;
+          qkv_epilogue64(ep, row, n_blk * BN + c, acc, rs, tile, lane);
+        } else {
+          if (row < M) epilogue64<KIND, bf16, DH>(ep, row, n_blk * BN + c, acc, rs);
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);

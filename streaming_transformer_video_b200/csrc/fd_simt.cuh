@@ -86,14 +86,20 @@ struct EmbedParams {
   int* status;            // device status word (bounds-checked build)
 };
 
-constexpr int kEmbedTok = 8;
+constexpr int kEmbedTok = 16;          // tokens per CTA
+constexpr int kEmbedThreads = 256;     // each thread: 4 consecutive columns of every token
 
-// One CTA = kEmbedTok tokens; thread d handles columns d, d+256, ...
-// Sums of squares per 32-column chunk come from a warp reduction (each warp
-// owns whole 32-column chunks).
+// One CTA = kEmbedTok tokens x all D columns (D a multiple of 32). The
+// gathered latent values of the CTA's tokens sit in shared memory, channel-
+// major so that one 16-byte broadcast read serves four tokens;
+// thread i accumulates columns 4i .. 4i+3 of every token in registers, reading
+// one 16-byte row of the transposed projection per input channel, so each
+// weight load feeds kEmbedTok x 4 FMAs and every store of x (fp32 and storage
+// type) is a contiguous run across the warp. The sum of squares of each
+// 32-column chunk comes from the 8 lanes that own it.
 template <typename T>
-__global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
-  extern __shared__ float u[];                          // [kEmbedTok][c_in]
+__global__ void __launch_bounds__(kEmbedThreads) embed_kernel(EmbedParams p) {
+  extern __shared__ float u[];                          // [c_in][kEmbedTok]
   griddep_wait();
   griddep_launch();
   const int n0 = blockIdx.x * kEmbedTok;
@@ -108,32 +114,56 @@ __global__ void __launch_bounds__(256) embed_kernel(EmbedParams p) {
       const size_t off = ((size_t(b) * p.C + c) * p.Hl + i * p.p + dy) * p.Wl + j * p.p + dx;
       if (FD_IN_BOUNDS(i * p.p + dy < p.Hl && j * p.p + dx < p.Wl, p.status))
         v = p.latent_bf16 ? __bfloat162float(static_cast<const bf16*>(p.latent)[off])
-                        : static_cast<const float*>(p.latent)[off];
+                          : static_cast<const float*>(p.latent)[off];
     }
-    u[idx] = v;
+    u[ch * kEmbedTok + tk] = v;
   }
   __syncthreads();
-  const int parts = p.D / 32;
-  for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
-    float acc[kEmbedTok];
-    const float bd = __ldg(p.b + d);
+  const int parts = p.D / 32, lane = threadIdx.x & 31;
+  // column groups of 4 kEmbedThreads; a lane past D computes on column 0 and
+  // stores nothing, so every lane takes part in the shuffles
+  for (int c0 = 0; c0 < p.D; c0 += 4 * kEmbedThreads) {
+    const int col = c0 + 4 * threadIdx.x;
+    if (c0 + 4 * (threadIdx.x & ~31) >= p.D) break;      // whole warp past D
+    const bool active = col < p.D;
+    const int cc = active ? col : 0;
+    const float4 bd = __ldg(reinterpret_cast<const float4*>(p.b + cc));
+    float4 acc[kEmbedTok];
 #pragma unroll
     for (int t = 0; t < kEmbedTok; ++t) acc[t] = bd;
+    const float4* w = reinterpret_cast<const float4*>(p.wT + cc);
+    const int wstride = p.D / 4;
+#pragma unroll 4
     for (int ch = 0; ch < p.c_in; ++ch) {
-      const float w = __ldg(p.wT + size_t(ch) * p.D + d);
+      const float4 wv = __ldg(w + size_t(ch) * wstride);
+      const float4* uc = reinterpret_cast<const float4*>(u + ch * kEmbedTok);   // broadcast
 #pragma unroll
-      for (int t = 0; t < kEmbedTok; ++t) acc[t] = fmaf(u[t * p.c_in + ch], w, acc[t]);
+      for (int t4 = 0; t4 < kEmbedTok / 4; ++t4) {
+        const float4 a4 = uc[t4];
+        const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int t = 4 * t4 + k;
+          acc[t].x = fmaf(a[k], wv.x, acc[t].x);
+          acc[t].y = fmaf(a[k], wv.y, acc[t].y);
+          acc[t].z = fmaf(a[k], wv.z, acc[t].z);
+          acc[t].w = fmaf(a[k], wv.w, acc[t].w);
+        }
+      }
     }
 #pragma unroll
     for (int t = 0; t < kEmbedTok; ++t) {
       const int n = n0 + t;
-      float s = acc[t] * acc[t];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (n < p.M) {
-        p.x32[size_t(n) * p.D + d] = acc[t];
-        static_cast<T*>(p.xb)[size_t(n) * p.D + d] = from_f<T>(acc[t]);
-        if ((threadIdx.x & 31) == 0) p.ssq[size_t(n) * parts + d / 32] = s;
+      const float4 o = acc[t];
+      float s = o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (active && n < p.M) {
+        *reinterpret_cast<float4*>(p.x32 + size_t(n) * p.D + col) = o;
+        const float v[4] = {o.x, o.y, o.z, o.w};
+        store_quad<T>(static_cast<T*>(p.xb) + size_t(n) * p.D + col, v);
+        if ((lane & 7) == 0) p.ssq[size_t(n) * parts + col / 32] = s;
       }
     }
   }

@@ -7,18 +7,23 @@ with the same scales, round to nearest even and take each rounding decision
 on a float32 product.
 
 Sharp check (test_block_mlp_on_identical_inputs): each block's O-projection
-+ MLP kernels run on a residual stream given to both sides bit-identically,
-so the E4M3 codes of the MLP input agree exactly; relative L2 of the MLP
-output <= 1e-4.
++ MLP kernels run on a residual stream given to both sides bit-identically;
+the E4M3 codes of RMSNorm(x) and of the hidden activation can then differ
+only where a float32 value sits within rounding noise of an E4M3 boundary;
+relative L2 of the MLP output <= 1e-4.
 
-End to end, the float32/bf16 arithmetic before each decision differs between
-the two sides, and E4M3 (3 fraction bits) turns such differences into
-one-step code changes: measured on the oracle alone, a 1e-4 relative
-perturbation of the latents moves its FP8 output by 1.2e-2 (small config),
-2.4e-2 (paper head) and 3.7e-2 (480p, 12 blocks) relative L2, max abs up to
-0.21, against 9e-5 without FP8. The GPU's end-to-end distance to the oracle
-is 1.1-1.7 times that. Tolerance, re-stated for FP8 configurations: output
-relative L2 <= 6e-2 and max abs <= 0.4. The GPU's FP8 result must also move
+End to end, the float32/bf16 arithmetic before each quantization point
+differs between the two sides, and E4M3 (3 fraction bits) turns such
+differences into one-step code changes. Measured on the oracle alone, a 1e-4
+relative perturbation of the latents moves its FP8 output by 1.0e-2 (small
+config), 1.2e-2 (GQA ratio 8), 2.4e-2 (paper head) and 3.7e-2 (480p, 12
+blocks) relative L2, max abs up to 0.21, against 9e-5 without FP8. The GPU's
+end-to-end distance to the oracle is 1.05-1.9 times that (2.0e-2, 2.0e-2,
+3.2e-2, 3.9e-2; max abs up to 0.23). Tolerance for FP8 configurations,
+derived from the largest self-sensitivity (3.7e-2, 0.21) with about 35%
+margin: output relative L2 <= 5e-2 and max abs <= 0.3. The bf16 bounds
+(2e-2, 5e-2) cannot hold: the oracle itself moves further than that under a
+perturbation far below bf16 rounding. The GPU's FP8 result must also move
 away from its bf16 result by about as much as the oracle's FP8 result moves
 away from its unquantized one.
 
@@ -35,8 +40,8 @@ from gpu_util import errors, gpu_decode, oracle_decode, small_bf16
 
 pytestmark = pytest.mark.gpu
 
-FP8_REL_L2 = 6e-2
-FP8_MAX_ABS = 0.4
+FP8_REL_L2 = 5e-2
+FP8_MAX_ABS = 0.3
 
 
 @pytest.fixture(scope="module", autouse=True)
