@@ -37,11 +37,11 @@ DEFAULT_CONFIG = "1080p_wan22"
 
 # DRAM traffic of one attention launch (one block, full window) measured by
 # ncu (dram__bytes_read.sum + dram__bytes_write.sum), see
-# profiles/block_1080p_ncu_full.md. Keyed by the sha256 of the kernel source:
+# profiles/attention_1080p_ncu.md. Keyed by the sha256 of the kernel source:
 # when the kernel changes the figure no longer applies and is reported as null.
 NCU_ATTN_TRAFFIC = {
-    ("1080p_wan22", "97cf5174fe98f8189f7652838c6f3553b8488c727c340500335f57fb58ff6c60"):
-        164032512 + 57520384,
+    ("1080p_wan22", "18e75f4f177e79c8501a21f412c7d2c45390de89fd1d1f60ae0e490bc18ceb6b"):
+        163831040 + 57682944,
 }
 
 
@@ -303,6 +303,8 @@ def run_flashdec(args):
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     cfg = fd_synth.CONFIGS[args.config].replace(batch=args.batch)
+    if args.blocks > 0:
+        cfg = cfg.replace(n_blocks=args.blocks)
     td = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     weights = fd_synth.make_weights(cfg)
     n_frames = args.warmup + args.steps
@@ -491,6 +493,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=1,
                     help="video streams decoded together per step (each its own video)")
+    ap.add_argument("--blocks", type=int, default=0,
+                    help="profiling only: override the number of Transformer blocks "
+                         "(a shallower decoder of the same width, for short ncu captures; "
+                         "its line is not the workload's measurement)")
     ap.add_argument("--mlp-fp8", action="store_true",
                     help="FP8 E4M3 MLP GEMMs with static scales calibrated on the warm-up "
                          "frames by a bf16 handle that records the MLP ranges")

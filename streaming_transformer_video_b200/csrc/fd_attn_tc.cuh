@@ -19,7 +19,11 @@
 //   warps 2..5  softmax, one query row per thread: S row from TMEM, base-2
 //               online softmax with lazy rescaling (O is rescaled in TMEM only
 //               when the running max grows by more than 2^8), P packed to bf16
-//               and written over the S it came from
+//               and written over the S it came from. After the first tile, P
+//               is formed against the running reference before the tile's
+//               own max is known; the max (which only decides the rare
+//               rescale, after which P is formed again) then overlaps the
+//               exponentials instead of preceding them
 // TMEM columns: S buffer b (b < 3) at 64 b, with P(j) in the first 32 columns
 // of its buffer; O at 192. S runs up to three tiles ahead of the softmax,
 // whose only synchronisation per tile is the wait for S(j) and the arrival
@@ -122,6 +126,14 @@ __device__ __forceinline__ float exp_pack64(const float* x, float sc, float m, u
   }
   a0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
   return a0.x + a0.y;
+}
+
+__device__ __forceinline__ float tile_max64(const float* x) {
+  float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
+#pragma unroll
+  for (int c = 6; c < 62; c += 4) { m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]); }
+  m0 = max3(m0, x[62], x[63]);
+  return fmaxf(m0, m1);
 }
 
 struct TcAttnSmem {
@@ -277,18 +289,24 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
           *reinterpret_cast<uint16_t*>(vt + d * 128 + (((c >> 3) ^ (d & 7)) << 4) + (c & 7) * 2) = 0;
         fence_proxy_async_smem();
       }
-      float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
-#pragma unroll
-      for (int c = 6; c < 62; c += 4) { m0 = max3(m0, x[c], x[c + 1]); m1 = max3(m1, x[c + 2], x[c + 3]); }
-      m0 = max3(m0, x[62], x[63]);
-      const float mx = fmaxf(m0, m1) * sc;
-      bool rescale = false;
-      if (j == 0) m_ref = mx;
-      else if (mx > m_ref + 8.f) rescale = true;
-      const float corr = rescale ? ex2(m_ref - mx) : 1.f;
-      if (rescale) { m_ref = mx; l *= corr; }
       uint32_t pk[32];
-      l += exp_pack64(x, sc, m_ref, pk);
+      float lt = 0.f, mx;
+      if (j == 0) {
+        mx = tile_max64(x) * sc;
+        m_ref = mx;
+        lt = exp_pack64(x, sc, m_ref, pk);
+      } else {
+        lt = exp_pack64(x, sc, m_ref, pk);           // independent of the tile max
+        mx = tile_max64(x) * sc;
+      }
+      const bool rescale = j > 0 && mx > m_ref + 8.f;
+      const float corr = rescale ? ex2(m_ref - mx) : 1.f;
+      if (rescale) {                                 // rare: redo this row's P
+        m_ref = mx;
+        l *= corr;
+        lt = exp_pack64(x, sc, m_ref, pk);
+      }
+      l += lt;
       if (__any_sync(0xffffffffu, rescale)) {
         // O *= corr (rare): every earlier O += P V must have landed first
         const int jp = j - 1;

@@ -151,11 +151,13 @@ __global__ void __launch_bounds__(gemm_threads(KIND), 1)
       const int m_blk = tile / n_n, n_blk = tile - (tile / n_n) * n_n;
       const int buf = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      if (!mbar_wait_warp(&acc_full[buf], acc_phase, abort_flag, status)) break;
-      tc_fence_after();
+      // the RMSNorm row scale does not depend on the accumulator: its loads
+      // overlap the tile's main loop
       const int row = m_blk * 128 + quarter * 32 + lane;
       float rs = 1.f;
       if (epi_normed(KIND) && row < M && ep.ssq) rs = row_scale(ep, row);
+      if (!mbar_wait_warp(&acc_full[buf], acc_phase, abort_flag, status)) break;
+      tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + buf * BN;
 #pragma unroll 1
       for (int c = 64 * half; c < BN; c += 64 * kPerQuarter) {
