@@ -53,6 +53,13 @@ def is_paper(cfg) -> bool:
     return getattr(cfg, "head", "linear") == "paper"
 
 
+def refine_batched(cfg) -> bool:
+    """The library runs all r_t sub-frames through each refinement block in one
+    launch per kernel for bf16 storage with L_frm a multiple of 8 (the ring
+    layout the decoder reports through ring_layout), else one at a time."""
+    return is_paper(cfg) and cfg.dtype == "bf16" and cfg.L_frm % 8 == 0
+
+
 def describe(cfg) -> str:
     streams = f"{cfg.batch} video streams per step, " if getattr(cfg, "batch", 1) > 1 else ""
     head = (f"paper head (upsample x{cfg.r_t}, {cfg.n_refine} refinement blocks over "
@@ -69,11 +76,16 @@ def describe(cfg) -> str:
 def attn_flops_per_launch(cfg):
     """FLOPs of each attention launch of one steady-state frame, in launch
     order: the backbone blocks (window of W+1 frames), then with the paper
-    head r_t x n_refine refinement launches (window of r_t (W+1) sub-frames)."""
+    head the refinement launches (window of r_t (W+1) sub-frames): one per
+    block covering all r_t sub-frames, or r_t x n_refine of one sub-frame."""
     L, hd, B = cfg.L_frm, cfg.n_heads * cfg.head_dim, getattr(cfg, "batch", 1)
     out = [B * 4 * L * ((cfg.window + 1) * L) * hd] * cfg.n_blocks
     if is_paper(cfg):
-        out += [B * 4 * L * (cfg.r_t * (cfg.window + 1) * L) * hd] * (cfg.r_t * cfg.n_refine)
+        sub = B * 4 * L * (cfg.r_t * (cfg.window + 1) * L) * hd
+        if refine_batched(cfg):
+            out += [cfg.r_t * sub] * cfg.n_refine
+        else:
+            out += [sub] * (cfg.r_t * cfg.n_refine)
     return out
 
 
@@ -91,11 +103,26 @@ def kind_flops(cfg):
     return f
 
 
+def frame_kind_flops(cfg):
+    """FLOPs of each GEMM kind summed over the launches of one frame."""
+    k = kind_flops(cfg)
+    blocks = cfg.n_blocks + (cfg.r_t * cfg.n_refine if is_paper(cfg) else 0)
+    out = {n: blocks * k[n] for n in ("qkv", "oproj", "mlp_up", "mlp_down")}
+    out["embed"] = k["embed"]
+    if is_paper(cfg):
+        out.update(upsample=k["upsample"], spatial=cfg.r_t * k["spatial"],
+                   final=cfg.r_t * k["final"])
+    else:
+        out["final"] = k["final"]
+    return out
+
+
 def kernels_per_frame(cfg) -> int:
     per_block = 5 + (1 if getattr(cfg, "mlp_fp8", 0) else 0)   # FP8: + MLP-input quantization
     n = 2 + per_block * cfg.n_blocks                    # step_begin, embed, backbone
     if is_paper(cfg):
-        return n + 1 + cfg.r_t * (per_block * cfg.n_refine + 2)  # upsample, refinement, spatial MLP
+        sub = 1 if refine_batched(cfg) else cfg.r_t     # launches per refinement kernel
+        return n + 1 + sub * (per_block * cfg.n_refine + 2)  # upsample, refinement, spatial MLP
     return n + 1                                        # final
 
 
@@ -466,9 +493,10 @@ def run_flashdec(args):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
     }
-    for k, f in kind_flops(cfg).items():
+    # per kind: its FLOPs in one frame over its launches' time in the last frame
+    for k, f in frame_kind_flops(cfg).items():
         if k in kern and k != "embed":
-            line["kernels_tflops"][k] = f / (line["kernels_ms"][k] * 1e-3) / 1e12
+            line["kernels_tflops"][k] = f / (float(np.sum(kern[k])) * 1e-3) / 1e12
     # attention launches of the last frame of the breakdown pass, in launch order
     per_frame_attn = kern["attn"][-len(attn_fl):]
     line["kernels_tflops"]["attn"] = sum(attn_fl) / (sum(per_frame_attn) * 1e-3) / 1e12

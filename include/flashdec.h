@@ -12,8 +12,11 @@
  * the output head is the paper's own (Sec. 3.4): a Linear D -> r_t D splits
  * each latent frame into r_t sub-frames (Eq. 3), refinement blocks stream
  * those sub-frames one after another with the same rolling-cache mechanism
- * (ring of r_t (W+1) sub-frames), and a 2-layer MLP + PixelShuffle turns each
- * refined sub-frame into one pixel frame.
+ * (each sub-frame attends to the last r_t (W+1) sub-frames), and a 2-layer
+ * MLP + PixelShuffle turns each refined sub-frame into one pixel frame.
+ * With bf16 storage and L_frm a multiple of 8, all r_t sub-frames of a latent
+ * frame pass each refinement block in one launch per kernel, each with its
+ * own window of the ring (same results as one after another).
  *
  * Conventions of this library:
  *   - W (fd_config.window) counts PAST latent frames. The cache keeps the
@@ -91,7 +94,7 @@ typedef struct {
   int32_t head_mode;     /* 0: final RMSNorm + Linear D -> C r_t P^2 + unpatchify.
                             1: the paper's head (Sec. 3.4): Linear D -> r_t D
                             (Eq. 3) into r_t sub-frames, streamed through
-                            n_refine refinement blocks with a cache of r_t (W+1)
+                            n_refine refinement blocks with a window of r_t (W+1)
                             sub-frames, then RMSNorm, Linear D -> D, GELU,
                             Linear D -> C P^2 and PixelShuffle per sub-frame    */
   int32_t n_refine;      /* refinement blocks (head_mode 1; 1 .. 8)              */
@@ -246,7 +249,8 @@ FD_API fd_status_t fd_stream_frame_index(fd_handle* h, int b, int64_t* t_out);
 FD_API fd_status_t fd_device_bytes(fd_handle* h, size_t* bytes_out);
 
 /* Bytes of the ring caches alone: n_blocks * 2 * G * (W+1) L_frm * D_h * elt,
- * plus n_refine * 2 * G * r_t (W+1) L_frm * D_h * elt with head_mode 1. */
+ * plus, with head_mode 1, n_refine * 2 * G * S L_frm * D_h * elt where S is
+ * the refinement ring's slots times their copies (fd_debug_ring_layout). */
 FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 
 /*
@@ -258,12 +262,30 @@ FD_API fd_status_t fd_cache_bytes(fd_handle* h, size_t* bytes_out);
 FD_API fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float* host_dst);
 
 /*
+ * Test/debug: the ring layout of block `block` (as fd_debug_read_ring numbers
+ * blocks): *slots = frames (or sub-frames) it holds, frame f in slot f mod
+ * *slots; *copies = 1, or 2 when every slot is stored twice (slot s also at
+ * s + *slots). The backbone has W+1 slots and one copy. The refinement ring
+ * ([FD] Sec. 3.4 Step 2: each sub-frame attends to the last r_t (W+1)
+ * sub-frames) has r_t (W+1) slots and one copy when sub-frames go through it
+ * one at a time, and r_t (W+2) - 1 slots in two copies when all r_t
+ * sub-frames of a latent frame go through it in one launch: writing them then
+ * evicts no sub-frame an earlier one of the same frame still attends to, and
+ * every window is one contiguous run of the doubled ring. This layout is the
+ * library's own; the paper fixes only which sub-frames each one attends to.
+ * Errors: FD_ERR_BAD_HANDLE, FD_ERR_INVALID_ARG (block out of range, null output).
+ */
+FD_API fd_status_t fd_debug_ring_layout(fd_handle* h, int32_t block, int32_t* slots,
+                                        int32_t* copies);
+
+/*
  * Test/debug: copy ring slot `slot` of block `block`, video stream b
  * (0 <= b < batch), to host memory as fp32 [G][L_frm][D_h]. Blocks
  * 0 .. n_blocks-1 are the backbone (slots 0 .. W); with head_mode 1, blocks
- * n_blocks .. n_blocks + n_refine - 1 are the refinement blocks, whose ring
- * holds r_t (W+1) sub-frames (sub-frame s in slot s mod r_t (W+1), [FD]
- * Sec. 3.4 Step 2). kv as for fd_debug_read_slot. Synchronous.
+ * n_blocks .. n_blocks + n_refine - 1 are the refinement blocks, whose slots
+ * and copies fd_debug_ring_layout gives (slot < slots x copies; slot
+ * s + slots is the second copy of slot s). kv as for fd_debug_read_slot.
+ * Synchronous.
  */
 FD_API fd_status_t fd_debug_read_ring(fd_handle* h, int block, int b, int slot, int kv,
                                       float* host_dst);
@@ -317,9 +339,10 @@ FD_API fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_ho
  * *n_out = number of timed kernels per frame. Pass cap = 0 to query *n_out
  * only. Each replay of the frame graph overwrites the previous frame's times.
  */
-/* With head_mode 1 a frame runs, after the backbone: UPSAMPLE once, then per
- * sub-frame the refinement blocks' QKV .. MLP_DOWN kernels, SPATIAL (first
- * MLP layer) and FINAL (second layer + PixelShuffle). */
+/* With head_mode 1 a frame runs, after the backbone: UPSAMPLE once, then the
+ * refinement blocks' QKV .. MLP_DOWN kernels, SPATIAL (first MLP layer) and
+ * FINAL (second layer + PixelShuffle): once over all r_t sub-frames when the
+ * refinement ring has two copies (fd_debug_ring_layout), else per sub-frame. */
 typedef enum {
   FD_K_STEP_BEGIN = 0, FD_K_EMBED = 1, FD_K_QKV = 2, FD_K_ATTN = 3,
   FD_K_OPROJ = 4, FD_K_MLP_UP = 5, FD_K_MLP_DOWN = 6, FD_K_FINAL = 7,

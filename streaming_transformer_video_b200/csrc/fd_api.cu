@@ -166,10 +166,22 @@ struct KernelLaunch {
   int kind;
 };
 
+// TMA maps of the scratch buffers whose row count is that of the launch:
+// one latent frame (M = B L rows), or all r_t sub-frames of the paper head's
+// refinement blocks together (r_t M rows).
+struct RowMaps {
+  CUtensorMap q;            // Q [H][n_sub B][L][64]
+  CUtensorMap o;            // attention output [rows][H Dh]
+  CUtensorMap h;            // MLP hidden [rows][4D]
+  CUtensorMap hs;           // spatial MLP hidden [rows][D] (paper head)
+  CUtensorMap x8, h8;       // FP8 MLP operands [rows][D], [rows][4D]
+};
+
 // Where one Transformer block reads and writes: its residual stream (one
-// latent frame, or one sub-frame of the paper head) and its ring cache.
+// latent frame, one sub-frame of the paper head, or all r_t sub-frames at
+// once) and its ring cache.
 struct BlockIO {
-  float* x32;               // [M][D] fp32 residual stream (M = B L rows)
+  float* x32;               // [M][D] fp32 residual stream (M rows)
   void* xb;                 // [M][D] storage-type copy (A operand)
   float* ssq;               // [M][D/32] sums of squares of x32
   const CUtensorMap* tm_x;  // map of xb (bf16 path)
@@ -179,7 +191,13 @@ struct BlockIO {
   const CUtensorMap* tm_k;  // maps over all layers of kc / vtc (bf16 path)
   const CUtensorMap* tm_v;
   int layer;                // this block's layer inside kc / vtc
-  const FrameState* fs;     // stream 0's state of the (sub-)frame; stride fs_stride
+  const FrameState* fs;     // state of stream 0, first (sub-)frame; stride fs_stride
+  int M;                    // rows: n_sub sub-frames x B streams x L tokens
+  int n_sub;                // sub-frames in one launch (1, or r_t)
+  int kv_mirror;            // mirrored ring: rows between a key's two copies (0: none)
+  int n_layers;             // layers of the ring (slabs of tm_k / tm_v: n_layers B G)
+  int n_split;              // attention key splitting of this launch shape
+  const RowMaps* maps;      // row-count-dependent maps (bf16 path)
 };
 
 // An attention node of the frame graph, kept so that its scratch pointers can
@@ -213,13 +231,22 @@ struct fd_handle {
   int fp8 = 0;                      // 1: FP8 E4M3 MLP GEMMs
   int tok_h = 0, tok_w = 0, L = 0, c_in = 0, qkv = 0, dff = 0, c_out = 0;
   int B = 1, M = 0;                 // video streams; GEMM rows M = B L
-  int n_split = 1;                  // attention key splitting (1: off)
+  int n_split = 1;                  // attention key splitting (1: off), one latent frame
+  int n_split_ref = 1;              // the same for the batched refinement launches
+  size_t split_units_max = 0;       // largest attention launch with splitting: units
+  size_t split_rows_max = 0;        // and partial rows (units x n_split x 128)
   float *part_o = nullptr, *part_ml = nullptr;   // its partial results
   int* split_ctr = nullptr;
   int fs_stride = 1;                // FrameStates per stream: 1 (+ r_t, paper head)
   int kv_rows = 0, vt_pitch = 0, out_h = 0, out_w = 0, num_sms = 0;
   int device = -1;                  // the CUDA device the handle was created on
-  int rkv_rows = 0, rvt_pitch = 0;  // refinement ring: r_t (W+1) sub-frames
+  int rkv_rows = 0, rvt_pitch = 0;  // refinement ring rows: ref_slots (x2 if mirrored) L
+  // paper head: all r_t sub-frames pass each refinement block in one launch
+  // per kernel (ref_batch), over a mirrored ring of ref_slots = r_t (W+2) - 1
+  // sub-frames stored twice; otherwise sub-frame by sub-frame over a ring of
+  // ref_slots = r_t (W+1)
+  int ref_batch = 0, ref_slots = 0;
+  int RM = 0;                       // rows of the largest launch: r_t M (ref_batch) or M
   size_t k_bytes = 0, v_bytes = 0, rk_bytes = 0, rv_bytes = 0;
   size_t latent_elems = 0, out_elems = 0, io_elt = 0, elt = 0;
 
@@ -267,8 +294,9 @@ struct fd_handle {
   bool user_pending = true; // caller-stream work since the last host call
 
   // TMA maps (bf16 path)
-  CUtensorMap tm_xb{}, tm_o{}, tm_h{}, tm_q{}, tm_k{}, tm_v{}, tm_wout{};
-  CUtensorMap tm_rk{}, tm_rv{}, tm_wup{}, tm_wsp1{}, tm_hs{}, tm_x8{}, tm_h8{};
+  CUtensorMap tm_xb{}, tm_k{}, tm_v{}, tm_wout{};
+  CUtensorMap tm_rk{}, tm_rv{}, tm_wup{}, tm_wsp1{}, tm_xs_all{};
+  RowMaps rm_frame{}, rm_ref{};        // M rows; r_t M rows (ref_batch)
   std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_w1, tm_w2, tm_xs;
 
   // graph
@@ -422,9 +450,9 @@ struct fd_handle {
   fd_status_t add_post_attention(int wi, const BlockIO& io);
   fd_status_t add_norm_quant(const BlockIO& io, int wi, float q_inv, unsigned* rec);
   EpiParams base_epi(const BlockIO& io) const;
-  size_t split_units() const { return size_t((L + 127) / 128) * cfg.n_heads * B; }
   BlockIO backbone_io(int layer);
   BlockIO subframe_io(int tau, int layer);
+  BlockIO refine_io(int layer);
 };
 
 namespace {
@@ -485,8 +513,9 @@ const void* simt_gemm_fn(int dh) {
 
 EpiParams fd_handle::base_epi(const BlockIO& io) const {
   EpiParams e{};
-  e.M = M;
+  e.M = io.M;
   e.L = L;
+  e.B = B;
   e.fs_stride = fs_stride;
   e.out_stride = out_elems;
   e.ssq = io.ssq;
@@ -503,6 +532,7 @@ EpiParams fd_handle::base_epi(const BlockIO& io) const {
   e.Dh = cfg.head_dim;
   e.kv_rows = io.kv_rows;
   e.vt_pitch = io.vt_pitch;
+  e.kv_mirror = io.kv_mirror;
   e.kv_norm = cfg.kv_norm;
   e.fs = io.fs;
   e.rope_row = rope_row;
@@ -522,15 +552,25 @@ EpiParams fd_handle::base_epi(const BlockIO& io) const {
 }
 
 BlockIO fd_handle::backbone_io(int layer) {
-  return BlockIO{x32, xb, ssq, &tm_xb, kc, vtc, kv_rows, vt_pitch, &tm_k, &tm_v, layer, fs};
+  return BlockIO{x32, xb, ssq, &tm_xb, kc, vtc, kv_rows, vt_pitch, &tm_k, &tm_v, layer, fs,
+                 M, 1, 0, cfg.n_blocks, n_split, &rm_frame};
 }
 
+// Sub-frame tau of the paper head through refinement layer `layer` alone.
 BlockIO fd_handle::subframe_io(int tau, int layer) {
   const size_t rows = size_t(tau) * M;
   const int D = cfg.d_model;
   return BlockIO{xs32 + rows * D, static_cast<char*>(xsb) + rows * D * elt,
                  xss + rows * (D / 32), bf ? &tm_xs[tau] : &tm_xb, rkc, rvtc, rkv_rows,
-                 rvt_pitch, &tm_rk, &tm_rv, layer, fs + 1 + tau};
+                 rvt_pitch, &tm_rk, &tm_rv, layer, fs + 1 + tau,
+                 M, 1, 0, cfg.n_refine, n_split, &rm_frame};
+}
+
+// All r_t sub-frames of the paper head through refinement layer `layer` in one
+// launch per kernel (rows (tau B + b) L + n of xs), over the mirrored ring.
+BlockIO fd_handle::refine_io(int layer) {
+  return BlockIO{xs32, xsb, xss, &tm_xs_all, rkc, rvtc, rkv_rows, rvt_pitch, &tm_rk, &tm_rv,
+                 layer, fs + 1, RM, cfg.r_t, ref_slots * L, cfg.n_refine, n_split_ref, &rm_ref};
 }
 
 // Kernel arguments must outlive the graph's construction; cudaGraphAddKernelNode
@@ -539,6 +579,7 @@ fd_status_t fd_handle::add_gemm(int kind, int fd_kind, const CUtensorMap& tmA, c
                                 const CUtensorMap& tmB, const void* B, int N, int K, EpiParams ep,
                                 cudaGraphNode_t* node, bool f8) {
   ep.N = N;
+  const int M = ep.M;
   KernelLaunch k{};
   if (bf) {
     int bn = 0;
@@ -615,9 +656,10 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.H = H;
     ap.G = G;
     ap.B = B;
+    ap.n_sub = io.n_sub;
     ap.fs_stride = fs_stride;
     ap.layer = io.layer;
-    ap.n_split = n_split;
+    ap.n_split = io.n_split;
     ap.part_o = part_o;
     ap.part_ml = part_ml;
     ap.counter = split_ctr;
@@ -625,15 +667,15 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.fs = io.fs;
     ap.status = status;
     ap.kv_rows = io.kv_rows;
-    ap.n_slabs = (io.kv_rows == kv_rows ? cfg.n_blocks : cfg.n_refine) * B * G;
+    ap.n_slabs = io.n_layers * B * G;
     // one 128-query tile per CTA, two CTAs per SM (measured faster than two
     // query tiles sharing one CTA, and than three CTAs with single-buffered S)
     using A = TcAttnSmem;
     const void* f = reinterpret_cast<const void*>(&tc_attn_kernel);
     FD_CUDA(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, A::kAlloc));
-    KernelLaunch k{f, dim3((L + 127) / 128, H, B * n_split), dim3(A::kThreads), size_t(A::kAlloc),
-                   FD_K_ATTN};
-    CUtensorMap a = tm_q, b = *io.tm_k, c = *io.tm_v;
+    KernelLaunch k{f, dim3((L + 127) / 128, H, io.n_sub * B * io.n_split), dim3(A::kThreads),
+                   size_t(A::kAlloc), FD_K_ATTN};
+    CUtensorMap a = io.maps->q, b = *io.tm_k, c = *io.tm_v;
     void* args[] = {&a, &b, &c, &ap};
     AttnNode an;
     FD_TRY(add_kernel(k, args, &an.node));
@@ -677,7 +719,8 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
     // output projection + residual (x32 and its sums of squares only)
     e = base_epi(io);
     e.bias = bo[wi];
-    FD_TRY(add_gemm(EPI_RESID_Q, FD_K_OPROJ, tm_o, o, tm_wo[wi], wo[wi], D, H * Dh, e, nullptr));
+    FD_TRY(add_gemm(EPI_RESID_Q, FD_K_OPROJ, io.maps->o, o, tm_wo[wi], wo[wi], D, H * Dh, e,
+                    nullptr));
     // the MLP-up's input: x8 = e4m3(RMSNorm(x) / s_a)
     FD_TRY(add_norm_quant(io, wi, float(1.0 / double(s_a[wi])), nullptr));
     // FP8 MLP up: h = GELU((x8 W1q^T) s_a s_w1 + b_1) stored as e4m3(h / s_h)
@@ -686,20 +729,20 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
     e.hout = hb;
     e.acc_scale = float(double(s_a[wi]) * double(s_w1[wi]));
     e.q_inv = float(1.0 / double(s_h[wi]));
-    FD_TRY(add_gemm(EPI_GELU_Q, FD_K_MLP_UP, tm_x8, x8, tm_w1[wi], w1[wi], dff, D, e, nullptr,
-                    true));
+    FD_TRY(add_gemm(EPI_GELU_Q, FD_K_MLP_UP, io.maps->x8, x8, tm_w1[wi], w1[wi], dff, D, e,
+                    nullptr, true));
     // FP8 MLP down + residual: x += (h8 W2q^T) s_h s_w2 + b_2
     e = base_epi(io);
     e.bias = b2[wi];
     e.acc_scale = float(double(s_h[wi]) * double(s_w2[wi]));
-    return add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h8, hb, tm_w2[wi], w2[wi], D, dff, e, nullptr,
-                    true);
+    return add_gemm(EPI_RESID, FD_K_MLP_DOWN, io.maps->h8, hb, tm_w2[wi], w2[wi], D, dff, e,
+                    nullptr, true);
   }
   // output projection + residual
   e = base_epi(io);
   e.bias = bo[wi];
-  FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, tm_o, o, bf ? tm_wo[wi] : tm_o, wo[wi], D, H * Dh, e,
-                  nullptr));
+  FD_TRY(add_gemm(EPI_RESID, FD_K_OPROJ, io.maps->o, o, bf ? tm_wo[wi] : io.maps->o, wo[wi], D,
+                  H * Dh, e, nullptr));
   // calibration: max |RMSNorm(x)| entering the MLP
   if (amax) FD_TRY(add_norm_quant(io, wi, 1.f, amax + 2 * wi));
   // MLP up + GELU
@@ -712,8 +755,8 @@ fd_status_t fd_handle::add_post_attention(int wi, const BlockIO& io) {
   // MLP down + residual
   e = base_epi(io);
   e.bias = b2[wi];
-  return add_gemm(EPI_RESID, FD_K_MLP_DOWN, tm_h, hb, bf ? tm_w2[wi] : tm_h, w2[wi], D, dff, e,
-                  nullptr);
+  return add_gemm(EPI_RESID, FD_K_MLP_DOWN, io.maps->h, hb, bf ? tm_w2[wi] : io.maps->h, w2[wi],
+                  D, dff, e, nullptr);
 }
 
 // RMSNorm(x) of the MLP's input (gain of block wi): its E4M3 image
@@ -725,12 +768,12 @@ fd_status_t fd_handle::add_norm_quant(const BlockIO& io, int wi, float q_inv, un
   np.g = g2[wi];
   np.x8 = rec ? nullptr : static_cast<uint8_t*>(x8);
   np.amax = rec;
-  np.M = M;
+  np.M = io.M;
   np.D = cfg.d_model;
   np.inv_d = 1.f / float(cfg.d_model);
   np.eps = cfg.norm_eps;
   np.q_inv = q_inv;
-  KernelLaunch k{reinterpret_cast<const void*>(&mlp_norm_quant_kernel), dim3((M + 7) / 8),
+  KernelLaunch k{reinterpret_cast<const void*>(&mlp_norm_quant_kernel), dim3((io.M + 7) / 8),
                  dim3(256), 0, FD_K_MLP_NORM};
   void* args[] = {&np};
   return add_kernel(k, args);
@@ -749,8 +792,9 @@ fd_status_t fd_handle::build_graph() {
     long long* c = ctr;
     FrameState* f = fs;
     int W = cfg.window, pairs = cfg.head_dim / 8, n_sub = paper ? cfg.r_t : 0, nb = B;
+    int sub_cap = paper ? ref_slots : 1, sub_mirror = ref_batch;
     const double* fr = inv_freq_t;
-    void* args[] = {&c, &f, &W, &pairs, &fr, &n_sub, &nb};
+    void* args[] = {&c, &f, &W, &pairs, &fr, &n_sub, &nb, &sub_cap, &sub_mirror};
     FD_TRY(add_kernel(k, args));
   }
   // embed
@@ -806,30 +850,40 @@ fd_status_t fd_handle::build_graph() {
     FD_TRY(add_gemm(EPI_UP, FD_K_UPSAMPLE, tm_xb, xb, bf ? tm_wup : tm_xb, wup, cfg.r_t * D, D, e,
                     nullptr));
     const int c_px = cfg.out_ch * cfg.px_per_token * cfg.px_per_token;
-    for (int tau = 0; tau < cfg.r_t; ++tau) {
-      // refinement blocks: sub-frame t r_t + tau in the ring of r_t (W+1)
-      for (int l = 0; l < cfg.n_refine; ++l) FD_TRY(add_block(cfg.n_blocks + l, subframe_io(tau, l)));
-      // spatial MLP layer 1: GELU(RMSNorm(xs) sp1_w^T + sp1_b) -> hidden [M][D]
-      const BlockIO io = subframe_io(tau, 0);
-      e = base_epi(io);
-      e.bias = bsp1;
-      e.hout = hb;
+    // spatial MLP (layer 1: GELU(RMSNorm(xs) sp1_w^T + sp1_b) -> hidden; layer
+    // 2 + PixelShuffle into pixel frames (c, tau), no norm) of the rows of io
+    auto spatial = [&](const BlockIO& io, int tau) -> fd_status_t {
+      EpiParams es = base_epi(io);
+      es.bias = bsp1;
+      es.hout = hb;
       FD_TRY(add_gemm(EPI_GELU, FD_K_SPATIAL, *io.tm_x, io.xb, bf ? tm_wsp1 : *io.tm_x, wsp1, D,
-                      D, e, nullptr));
-      // layer 2 + PixelShuffle into pixel frames (c, tau), no norm
+                      D, es, nullptr));
       OutNode on;
       on.p = base_epi(io);
       on.p.bias = bout;
       on.p.ssq = nullptr;
       on.p.out = out_stage[0];
       on.p.pl_mul = cfg.r_t;
-      on.p.pl_add = tau;
-      on.tmA = bf ? tm_hs : tm_xb;
+      on.p.pl_add = tau;                  // 0 for a batched launch: tau comes from the row
+      on.tmA = bf ? io.maps->hs : tm_xb;
       on.A = hb;
       on.tmB = bf ? tm_wout : tm_xb;
       on.B = wout;
       on.K = D;
-      FD_TRY(add_out_gemm(on, c_px));
+      return add_out_gemm(on, c_px);
+    };
+    if (ref_batch) {
+      // every refinement block once over all r_t sub-frames (r_t M rows), then
+      // the spatial MLP over all of them
+      for (int l = 0; l < cfg.n_refine; ++l) FD_TRY(add_block(cfg.n_blocks + l, refine_io(l)));
+      FD_TRY(spatial(refine_io(0), 0));
+    } else {
+      for (int tau = 0; tau < cfg.r_t; ++tau) {
+        // refinement blocks: sub-frame t r_t + tau in the ring of r_t (W+1)
+        for (int l = 0; l < cfg.n_refine; ++l)
+          FD_TRY(add_block(cfg.n_blocks + l, subframe_io(tau, l)));
+        FD_TRY(spatial(subframe_io(tau, 0), tau));
+      }
     }
   }
   cur_out = out_stage[0];
@@ -902,9 +956,12 @@ fd_status_t validate(const fd_config* c) {
       return fail(FD_ERR_UNSUPPORTED, "config: n_refine must be 1 .. 8 (got %d)", c->n_refine);
     if (c->r_t > 16)
       return fail(FD_ERR_UNSUPPORTED, "config: the paper head supports r_t <= 16 (got %d)", c->r_t);
-    if (L * c->r_t * (c->window + 1) > (1LL << 30))
-      return fail(FD_ERR_UNSUPPORTED, "config: refinement window of %lld tokens is too large",
-                  L * c->r_t * (c->window + 1));
+    // ring rows: r_t (W+1) sub-frames, or 2 (r_t (W+2) - 1) when mirrored
+    const long long ring = (c->dtype == FD_BF16 && L % 8 == 0)
+                               ? 2LL * (c->r_t * (c->window + 2) - 1) * L
+                               : L * c->r_t * (c->window + 1);
+    if (ring > (1LL << 30))
+      return fail(FD_ERR_UNSUPPORTED, "config: refinement ring of %lld tokens is too large", ring);
   }
   return FD_OK;
 }
@@ -929,8 +986,16 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   h->c_out = c.out_ch * c.r_t * c.px_per_token * c.px_per_token;
   h->kv_rows = (c.window + 1) * h->L;
   h->vt_pitch = int(round_up(size_t(h->kv_rows), 64));
-  h->rkv_rows = c.r_t * (c.window + 1) * h->L;
+  // paper head, bf16: the r_t sub-frames go through each refinement block in
+  // one launch per kernel, over a mirrored ring (every window a contiguous key
+  // range). The TMA load of the transposed values starts at key win * L, which
+  // must be a multiple of 8 (16 bytes), hence L % 8 == 0; otherwise, and on
+  // the fp32 path, sub-frame by sub-frame.
+  h->ref_batch = h->paper && h->bf && h->L % 8 == 0;
+  h->ref_slots = h->ref_batch ? c.r_t * (c.window + 2) - 1 : c.r_t * (c.window + 1);
+  h->rkv_rows = (h->ref_batch ? 2 : 1) * h->ref_slots * h->L;
   h->rvt_pitch = int(round_up(size_t(h->rkv_rows), 64));
+  h->RM = h->ref_batch ? c.r_t * h->M : h->M;
   h->out_h = h->tok_h * c.px_per_token;
   h->out_w = h->tok_w * c.px_per_token;
   h->latent_elems = size_t(c.latent_ch) * c.grid_h * c.grid_w;
@@ -998,7 +1063,7 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   }
 
   // ---- ring caches: K [layers][B][G][rows][Dh], V^T [layers][B][G][Dh][pitch];
-  // backbone rows = (W+1) L, refinement rows = r_t (W+1) L
+  // backbone rows = (W+1) L, refinement rows = ref_slots L (x2 when mirrored)
   const int BG = h->B * G;
   h->k_bytes = size_t(NB) * BG * h->kv_rows * Dh * h->elt;
   h->v_bytes = size_t(NB) * BG * Dh * h->vt_pitch * h->elt;
@@ -1014,41 +1079,53 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
 
   // ---- scratch
   const size_t L = h->M;                 // every per-frame buffer holds B frames
-  FD_TRY(h->alloc(&h->x32, L * D * 4));
+  const size_t RM = h->RM;               // the buffers a batched refinement launch
+  FD_TRY(h->alloc(&h->x32, L * D * 4));  // uses hold its r_t M rows
   FD_TRY(h->alloc(&h->xb, L * D * h->elt));
   FD_TRY(h->alloc(&h->ssq, L * (D / 32) * 4));
-  FD_TRY(h->alloc(&h->q, size_t(H) * L * Dh * h->elt));
-  FD_TRY(h->alloc(&h->o, L * H * Dh * h->elt));
-  FD_TRY(h->alloc(&h->hb, L * h->dff * h->elt));
+  FD_TRY(h->alloc(&h->q, size_t(H) * RM * Dh * h->elt));
+  FD_TRY(h->alloc(&h->o, RM * H * Dh * h->elt));
+  FD_TRY(h->alloc(&h->hb, RM * h->dff * h->elt));
   if (h->paper) {
     FD_TRY(h->alloc(&h->xs32, size_t(c.r_t) * L * D * 4));
     FD_TRY(h->alloc(&h->xsb, size_t(c.r_t) * L * D * h->elt));
     FD_TRY(h->alloc(&h->xss, size_t(c.r_t) * L * (D / 32) * 4));
   }
-  if (h->fp8) FD_TRY(h->alloc(&h->x8, L * D));
+  if (h->fp8) FD_TRY(h->alloc(&h->x8, RM * D));
   if (c.record_mlp_amax) {
     h->n_amax = 2 * (NB + NR);
     FD_TRY(h->alloc(&h->amax, size_t(h->n_amax) * 4));
   }
-  // attention key splitting: chosen by the attention launch's fit to the CTA
-  // slots (2 per SM): est(s) = waves(s units) / s, plus 4% per extra split for
-  // the partial writes and the combine
+  // attention key splitting, per launch shape (one latent frame; all r_t
+  // sub-frames of a batched refinement block): chosen by the launch's fit to
+  // the CTA slots (2 per SM): est(s) = waves(s units) / s, plus 4% per extra
+  // split for the partial writes and the combine. One scratch serves both
+  // shapes (their launches never overlap), sized for the larger.
   if (h->bf) {
-    const long units = long((h->L + 127) / 128) * H * h->B;
     const long slots = 2L * h->num_sms;
-    h->n_split = c.attn_splits;
-    if (h->n_split == 0) {
-      double best = 1e30;
-      for (int sp = 1; sp <= 3; ++sp) {
-        const double est = double((units * sp + slots - 1) / slots) / sp * (1.0 + 0.04 * (sp - 1));
-        if (est < best - 1e-9) { best = est; h->n_split = sp; }
+    auto pick = [&](long units) {
+      int ns = c.attn_splits;
+      if (ns == 0) {
+        double best = 1e30;
+        for (int sp = 1; sp <= 3; ++sp) {
+          const double est = double((units * sp + slots - 1) / slots) / sp * (1.0 + 0.04 * (sp - 1));
+          if (est < best - 1e-9) { best = est; ns = sp; }
+        }
       }
-    }
-    if (h->n_split > 1) {
-      FD_TRY(h->alloc(&h->part_o, size_t(units) * h->n_split * 128 * 64 * 4));
-      FD_TRY(h->alloc(&h->part_ml, size_t(units) * h->n_split * 128 * 2 * 4));
-      FD_TRY(h->alloc(&h->split_ctr, size_t(units) * 4));
-      FD_CUDA(cudaMemset(h->split_ctr, 0, size_t(units) * 4));
+      if (ns > 1) {
+        h->split_units_max = std::max(h->split_units_max, size_t(units));
+        h->split_rows_max = std::max(h->split_rows_max, size_t(units) * ns * 128);
+      }
+      return ns;
+    };
+    const long units = long((h->L + 127) / 128) * H * h->B;
+    h->n_split = pick(units);
+    h->n_split_ref = h->ref_batch ? pick(units * c.r_t) : h->n_split;
+    if (h->split_rows_max > 0) {
+      FD_TRY(h->alloc(&h->part_o, h->split_rows_max * 64 * 4));
+      FD_TRY(h->alloc(&h->part_ml, h->split_rows_max * 2 * 4));
+      FD_TRY(h->alloc(&h->split_ctr, h->split_units_max * 4));
+      FD_CUDA(cudaMemset(h->split_ctr, 0, h->split_units_max * 4));
     }
   }
   FD_TRY(h->alloc(&h->ctr, size_t(h->B) * 8));
@@ -1097,41 +1174,57 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
   // ---- tensor maps (bf16 path)
   if (h->bf) {
     FD_TRY(make_tmap_2d(&h->tm_xb, h->xb, L, D, 128));
-    FD_TRY(make_tmap_2d(&h->tm_o, h->o, L, size_t(H) * Dh, 128));
-    FD_TRY(make_tmap_2d(&h->tm_h, h->hb, L, h->dff, 128));
-    auto bn_of = [&](int N, int kind = EPI_QKV, int K = 0) {
-      return uint32_t(gemm_bn(kind, h->M, N, K, h->num_sms));
+    // maps of the buffers whose rows are those of the launch: one latent frame
+    // (M rows), and for batched refinement all r_t sub-frames (r_t M rows)
+    auto row_maps = [&](RowMaps* rm, size_t rows, int n_sub) -> fd_status_t {
+      FD_TRY(make_tmap_2d(&rm->o, h->o, rows, size_t(H) * Dh, 128));
+      FD_TRY(make_tmap_2d(&rm->h, h->hb, rows, h->dff, 128));
+      if (h->paper) FD_TRY(make_tmap_2d(&rm->hs, h->hb, rows, D, 128));   // spatial hidden
+      if (h->fp8) {
+        FD_TRY(make_tmap_2d_e4m3(&rm->x8, h->x8, rows, D, 128));
+        FD_TRY(make_tmap_2d_e4m3(&rm->h8, h->hb, rows, h->dff, 128));   // hidden as E4M3
+      }
+      // Q [H][n_sub B][L_frm][64]: box 64 x 128 x 1 x 1; a stream's last tile reads zeros
+      const uint64_t Lf = uint64_t(h->L), nb = uint64_t(n_sub) * h->B;
+      const uint64_t dims[4] = {64, Lf, nb, uint64_t(H)};
+      const uint64_t str[3] = {64 * 2, Lf * 64 * 2, nb * Lf * 64 * 2};
+      const uint32_t box[4] = {64, 128, 1, 1};
+      return make_tmap(&rm->q, h->q, 4, dims, str, box);
+    };
+    FD_TRY(row_maps(&h->rm_frame, L, 1));
+    if (h->ref_batch) FD_TRY(row_maps(&h->rm_ref, RM, c.r_t));
+    // a weight map's box is the BN rows its GEMM's tile width takes, which
+    // depends on the launch's row count
+    auto bn_of = [&](size_t rows, int N, int kind = EPI_QKV, int K = 0) {
+      return uint32_t(gemm_bn(kind, int(rows), N, K, h->num_sms));
     };
     for (int l = 0; l < NB + NR; ++l) {
+      const size_t rows = l < NB ? L : RM;
       CUtensorMap m;
-      FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(h->qkv))); h->tm_wqkv.push_back(m);
-      FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(D, EPI_RESID, H * Dh)));
+      FD_TRY(make_tmap_2d(&m, h->wqkv[l], h->qkv, D, bn_of(rows, h->qkv))); h->tm_wqkv.push_back(m);
+      FD_TRY(make_tmap_2d(&m, h->wo[l], D, size_t(H) * Dh, bn_of(rows, D, EPI_RESID, H * Dh)));
       h->tm_wo.push_back(m);
       if (h->fp8) {
-        FD_TRY(make_tmap_2d_e4m3(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
-        FD_TRY(make_tmap_2d_e4m3(&m, h->w2[l], D, h->dff, bn_of(D, EPI_RESID, h->dff)));
+        FD_TRY(make_tmap_2d_e4m3(&m, h->w1[l], h->dff, D, bn_of(rows, h->dff))); h->tm_w1.push_back(m);
+        FD_TRY(make_tmap_2d_e4m3(&m, h->w2[l], D, h->dff, bn_of(rows, D, EPI_RESID, h->dff)));
         h->tm_w2.push_back(m);
       } else {
-        FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(h->dff))); h->tm_w1.push_back(m);
-        FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(D, EPI_RESID, h->dff)));
+        FD_TRY(make_tmap_2d(&m, h->w1[l], h->dff, D, bn_of(rows, h->dff))); h->tm_w1.push_back(m);
+        FD_TRY(make_tmap_2d(&m, h->w2[l], D, h->dff, bn_of(rows, D, EPI_RESID, h->dff)));
         h->tm_w2.push_back(m);
       }
     }
-    if (h->fp8) {
-      FD_TRY(make_tmap_2d_e4m3(&h->tm_x8, h->x8, L, D, 128));
-      FD_TRY(make_tmap_2d_e4m3(&h->tm_h8, h->hb, L, h->dff, 128));   // hidden as E4M3 [L][4D]
-    }
     const int n_out = h->paper ? c_px : h->c_out;
-    FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, n_out, D, bn_of(n_out)));
+    FD_TRY(make_tmap_2d(&h->tm_wout, h->wout, n_out, D, bn_of(h->paper ? RM : L, n_out)));
     if (h->paper) {
-      FD_TRY(make_tmap_2d(&h->tm_wup, h->wup, size_t(c.r_t) * D, D, bn_of(c.r_t * D)));
-      FD_TRY(make_tmap_2d(&h->tm_wsp1, h->wsp1, D, D, bn_of(D)));
-      FD_TRY(make_tmap_2d(&h->tm_hs, h->hb, L, D, 128));          // spatial hidden [L][D]
+      FD_TRY(make_tmap_2d(&h->tm_wup, h->wup, size_t(c.r_t) * D, D, bn_of(L, c.r_t * D)));
+      FD_TRY(make_tmap_2d(&h->tm_wsp1, h->wsp1, D, D, bn_of(RM, D)));
       for (int tau = 0; tau < c.r_t; ++tau) {
         CUtensorMap m;
         FD_TRY(make_tmap_2d(&m, static_cast<char*>(h->xsb) + size_t(tau) * L * D * 2, L, D, 128));
         h->tm_xs.push_back(m);
       }
+      if (h->ref_batch) FD_TRY(make_tmap_2d(&h->tm_xs_all, h->xsb, RM, D, 128));
       const uint64_t kd[3] = {64, uint64_t(h->rkv_rows), uint64_t(NR) * BG};
       const uint64_t ks[2] = {64 * 2, uint64_t(h->rkv_rows) * 64 * 2};
       const uint32_t kb[3] = {64, 64, 1};
@@ -1140,13 +1233,6 @@ fd_status_t create_impl(const fd_config* cfg, const fd_weights* w, fd_handle* h)
       const uint64_t vs[2] = {uint64_t(h->rvt_pitch) * 2, uint64_t(h->rvt_pitch) * 64 * 2};
       const uint32_t vb[3] = {64, 64, 1};
       FD_TRY(make_tmap(&h->tm_rv, h->rvtc, 3, vd, vs, vb));
-    }
-    {   // Q [H][B][L_frm][64]: box 64 x 128 x 1 x 1; a stream's last tile reads zeros
-      const uint64_t Lf = uint64_t(h->L);
-      const uint64_t dims[4] = {64, Lf, uint64_t(h->B), uint64_t(H)};
-      const uint64_t str[3] = {64 * 2, Lf * 64 * 2, uint64_t(h->B) * Lf * 64 * 2};
-      const uint32_t box[4] = {64, 128, 1, 1};
-      FD_TRY(make_tmap(&h->tm_q, h->q, 4, dims, str, box));
     }
     {   // K [NB*G][kv_rows][64]: box 64 dims x 64 keys x 1
       const uint64_t dims[3] = {64, uint64_t(h->kv_rows), uint64_t(NB) * BG};
@@ -1288,7 +1374,7 @@ fd_status_t fd_reset(fd_handle* h, void* stream) {
   FD_CUDA(cudaMemsetAsync(h->ctr, 0, size_t(h->B) * 8, s));
   FD_CUDA(cudaMemsetAsync(h->status, 0, 16, s));
   if (h->amax) FD_CUDA(cudaMemsetAsync(h->amax, 0, size_t(h->n_amax) * 4, s));
-  if (h->split_ctr) FD_CUDA(cudaMemsetAsync(h->split_ctr, 0, h->split_units() * 4, s));
+  if (h->split_ctr) FD_CUDA(cudaMemsetAsync(h->split_ctr, 0, h->split_units_max * 4, s));
   h->last_stream = s;
   return FD_OK;
 }
@@ -1460,12 +1546,25 @@ fd_status_t fd_debug_read_slot(fd_handle* h, int block, int slot, int kv, float*
   return FD_OK;
 }
 
+fd_status_t fd_debug_ring_layout(fd_handle* h, int block, int32_t* slots, int32_t* copies) {
+  if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_ring_layout: invalid handle");
+  const fd_config& c = h->cfg;
+  const int n_all = c.n_blocks + (h->paper ? c.n_refine : 0);
+  if (block < 0 || block >= n_all || !slots || !copies)
+    return fail(FD_ERR_INVALID_ARG, "fd_debug_ring_layout: bad block or null output");
+  const bool refine = h->paper && block >= c.n_blocks;
+  *slots = refine ? h->ref_slots : c.window + 1;
+  *copies = refine && h->ref_batch ? 2 : 1;
+  return FD_OK;
+}
+
 fd_status_t fd_debug_read_ring(fd_handle* h, int block, int b, int slot, int kv, float* host_dst) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_debug_read_ring: invalid handle");
   const fd_config& c = h->cfg;
   const bool refine = h->paper && block >= c.n_blocks;
   const int n_all = c.n_blocks + (h->paper ? c.n_refine : 0);
-  const int slots = refine ? c.r_t * (c.window + 1) : c.window + 1;
+  // a mirrored refinement ring keeps slot s at s and s + ref_slots
+  const int slots = refine ? h->ref_slots * (h->ref_batch ? 2 : 1) : c.window + 1;
   if (block < 0 || block >= n_all || b < 0 || b >= h->B || slot < 0 || slot >= slots ||
       (kv != 0 && kv != 1) || !host_dst)
     return fail(FD_ERR_INVALID_ARG, "fd_debug_read_ring: bad block/stream/slot/kv/dst");
@@ -1534,7 +1633,7 @@ fd_status_t fd_debug_poison(fd_handle* h, int32_t what, void* stream) {
     }
   }
   if ((what & FD_POISON_SPLIT_COUNTERS) && h->split_ctr)
-    FD_CUDA(cudaMemsetAsync(h->split_ctr, 0x7F, h->split_units() * 4, s));
+    FD_CUDA(cudaMemsetAsync(h->split_ctr, 0x7F, h->split_units_max * 4, s));
   h->last_stream = s;
   return FD_OK;
 }
@@ -1546,9 +1645,15 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   if (block < 0 || block >= n_all || !x_host || !out_host)
     return fail(FD_ERR_INVALID_ARG, "fd_debug_block_mlp: bad block or null buffer");
   FD_CUDA(cudaDeviceSynchronize());
+  // the block's own launch shape: a refinement block that runs all r_t
+  // sub-frames at once gets r_t M rows (the caller's M first, zeros after),
+  // so its kernels take the tile widths its weight maps were built for
+  const bool ref = h->ref_batch && block >= c.n_blocks;
+  const BlockIO io = ref ? h->refine_io(0) : h->backbone_io(0);
   const size_t n = size_t(h->M) * c.d_model;
-  FD_CUDA(cudaMemcpy(h->x32, x_host, n * 4, cudaMemcpyHostToDevice));
-  FD_CUDA(cudaMemset(h->o, 0, size_t(h->M) * c.n_heads * c.head_dim * h->elt));
+  if (ref) FD_CUDA(cudaMemset(io.x32, 0, size_t(io.M) * c.d_model * 4));
+  FD_CUDA(cudaMemcpy(io.x32, x_host, n * 4, cudaMemcpyHostToDevice));
+  FD_CUDA(cudaMemset(h->o, 0, size_t(io.M) * c.n_heads * c.head_dim * h->elt));
   // a one-off graph of the block's post-attention kernels on the backbone
   // stream; no timing events, no calibration records
   cudaGraph_t saved_graph = h->graph;
@@ -1565,7 +1670,7 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   h->last_is_kernel = false;
   h->cfg.kernel_timing = 0;
   h->amax = nullptr;
-  fd_status_t st = h->add_post_attention(block, h->backbone_io(0));
+  fd_status_t st = h->add_post_attention(block, io);
   h->graph = saved_graph;
   h->last_node = saved_last;
   h->last_is_kernel = saved_is_kernel;
@@ -1577,7 +1682,7 @@ fd_status_t fd_debug_block_mlp(fd_handle* h, int block, const float* x_host, flo
   if (st == FD_OK && e == cudaSuccess) e = cudaGraphLaunch(ex, nullptr);
   if (st == FD_OK && e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
   if (st == FD_OK && e == cudaSuccess)
-    e = cudaMemcpy(out_host, h->x32, n * 4, cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(out_host, io.x32, n * 4, cudaMemcpyDeviceToHost);
   if (ex) cudaGraphExecDestroy(ex);
   cudaGraphDestroy(g);
   if (st == FD_OK && e != cudaSuccess) {
@@ -1612,11 +1717,13 @@ extern "C" {
 fd_status_t fd_decode_frame_static_scratch(fd_handle* h, const void* latent, void* out,
                                            void* stream) {
   if (!valid_handle(h)) return fail(FD_ERR_BAD_HANDLE, "fd_decode_frame_static_scratch: invalid handle");
-  if (h->n_split == 1 || h->attn_nodes.empty())       // this handle's attention uses no scratch
+  if (h->split_rows_max == 0 || h->attn_nodes.empty())   // this handle's attention uses no scratch
     return fd_decode_frame(h, latent, out, stream);
-  const size_t units = h->split_units();
-  const size_t o_bytes = units * h->n_split * 128 * 64 * 4;
-  const size_t ml_bytes = units * h->n_split * 128 * 2 * 4;
+  // the largest attention launch shape with key splitting (one latent frame,
+  // or all sub-frames of a batched refinement block)
+  const size_t units = h->split_units_max;
+  const size_t o_bytes = h->split_rows_max * 64 * 4;
+  const size_t ml_bytes = h->split_rows_max * 2 * 4;
   const size_t need = kStaticCtrBytes + round_up(o_bytes, 256) + ml_bytes;
   if (units * 4 > kStaticCtrBytes || need > kStaticScratchBytes)
     return fail(FD_ERR_UNSUPPORTED,

@@ -2,12 +2,16 @@
 //
 // Paper Sec. 3.3: the current frame's queries attend, with no mask, to every
 // cached key of the window (itself plus W past frames). Keys of ring slot s
-// are stored at rows [s*L, (s+1)*L) of the block's cache, so the valid keys
-// are always the contiguous range [0, n_valid*L) and softmax, being
-// invariant to the order of keys, needs no slot bookkeeping.
+// are stored at rows [s*L, (s+1)*L) of the block's cache, so the window's keys
+// are the contiguous range [win*L, (win + n_valid)*L) of the frame state
+// (win = 0 except in a mirrored ring, where every slot is stored twice) and
+// softmax, being invariant to the order of keys, needs no slot bookkeeping.
 //
 // One CTA = one head x 128 queries of one video stream (blockIdx.z; each
 // stream has its own frame state and cache slab); 192 threads, 2 CTAs per SM.
+// A launch may cover n_sub sub-frames of the paper head's refinement blocks
+// at once: blockIdx.z / n_split = tau * B + b picks sub-frame tau of stream b,
+// with its own frame state (and so its own key window in the shared ring).
 // Keys are consumed in tiles of 64.
 //   warp 0      TMA: Q once, then per stage K (64 keys x 64) and the
 //               transposed V (64 dims x 64 keys)
@@ -45,15 +49,16 @@
 namespace fd {
 
 struct TcAttnParams {
-  void* o;            // [B][L][H*64] bf16
+  void* o;            // [n_sub][B][L][H*64] bf16
   int L, H, G;
   int B;              // video streams
+  int n_sub;          // sub-frames per launch (1, or r_t for a whole refinement block)
   int layer;          // block index: cache map slab (layer * B + stream) * G + g
   int fs_stride;      // FrameStates per stream
   float scale_log2;   // log2(e) / sqrt(64)
-  const FrameState* fs;
+  const FrameState* fs;  // state of stream b, sub-frame tau: fs[b * fs_stride + tau]
   int* status;
-  // key splitting (n_split 1: off); unit = (stream * H + head) * gridDim.x + query tile
+  // key splitting (n_split 1: off); unit = ((tau * B + b) * H + head) * gridDim.x + query tile
   int n_split;
   float* part_o;      // [unit][n_split][128][64] unnormalised O
   float* part_ml;     // [unit][n_split][128][2] running max (log2 domain), sum
@@ -175,7 +180,8 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = blockIdx.x * 128, h = blockIdx.y;
-  const int bs = blockIdx.z / p.n_split, split = blockIdx.z - bs * p.n_split;
+  const int bq = blockIdx.z / p.n_split, split = blockIdx.z - bq * p.n_split;
+  const int bs = bq % p.B, tau = bq / p.B;            // video stream, sub-frame
   const int g = h / (p.H / p.G);
   const int lg = (p.layer * p.B + bs) * p.G + g;
 
@@ -197,8 +203,18 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
   const uint32_t tmem_base = *tmem_slot;
   griddep_wait();                                 // Q, K, V and the frame state
   griddep_launch();
-  int n_keys = p.fs[size_t(bs) * p.fs_stride].n_valid * p.L;
-  if (!FD_IN_BOUNDS(n_keys <= p.kv_rows && lg < p.n_slabs, p.status)) n_keys = 0;
+  const FrameState& fst = p.fs[size_t(bs) * p.fs_stride + tau];
+  int n_keys = fst.n_valid * p.L;
+  const int key0 = fst.win * p.L;                 // first key row of the window
+  if (!FD_IN_BOUNDS(key0 + n_keys <= p.kv_rows && lg < p.n_slabs && tau < p.n_sub, p.status))
+    n_keys = 0;
+  // the V^T tile's inner coordinate must be 16-byte aligned: a window start
+  // off that grid (never produced by the host, which mirrors only rings with
+  // L % 8 == 0) is refused rather than loaded
+  if (key0 & 7) {
+    if (threadIdx.x == 0) report_status(p.status, FD_ERR_BOUNDS);
+    n_keys = 0;
+  }
   const int n_kt_all = (n_keys + 63) / 64;
   // this CTA's key tiles: [j0, j0 + n_kt) (all of them without splitting)
   const int j0 = split * n_kt_all / p.n_split;
@@ -207,14 +223,14 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
   if (warp == 0) {
     if (lane == 0) {                                       // ---- TMA producer
       mbar_arrive_expect_tx(q_full, 16384);
-      tma_load_4d(smem + S::kQ, &tmQ, 0, q0, bs, h, q_full);
+      tma_load_4d(smem + S::kQ, &tmQ, 0, q0, bq, h, q_full);
       for (int j = 0; j < n_kt; ++j) {
         const int st = j % ST;
         if (!mbar_wait(&kv_empty[st], ((j / ST) & 1) ^ 1, abort_flag, p.status)) break;
         uint8_t* kv = smem + S::kKV + st * S::kKVStage;
         mbar_arrive_expect_tx(&kv_full[st], S::kKVStage);
-        tma_load_3d(kv, &tmK, 0, (j0 + j) * 64, lg, &kv_full[st]);
-        tma_load_3d(kv + 8192, &tmV, (j0 + j) * 64, 0, lg, &kv_full[st]);
+        tma_load_3d(kv, &tmK, 0, key0 + (j0 + j) * 64, lg, &kv_full[st]);
+        tma_load_3d(kv + 8192, &tmV, key0 + (j0 + j) * 64, 0, lg, &kv_full[st]);
       }
     }
   } else if (warp == 1) {
@@ -352,12 +368,12 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
         const float inv = 1.f / l;
 #pragma unroll
         for (int c = 0; c < 64; ++c) v[c] *= inv;
-        store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
+        store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bq) * p.L + row) * p.H * 64 +
                                 size_t(h) * 64, v);
       }
-    } else if (FD_IN_BOUNDS(bs < p.B && split < p.n_split, p.status)) {   // uniform per CTA
+    } else if (FD_IN_BOUNDS(bq < p.B * p.n_sub && split < p.n_split, p.status)) {   // uniform per CTA
       // this key range's partial result
-      const size_t unit = (size_t(bs) * p.H + h) * gridDim.x + blockIdx.x;
+      const size_t unit = (size_t(bq) * p.H + h) * gridDim.x + blockIdx.x;
       const size_t prow = (unit * p.n_split + split) * 128 + r;
       float4* po = reinterpret_cast<float4*>(p.part_o + prow * 64);
 #pragma unroll
@@ -397,7 +413,7 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
           const float inv = 1.f / lsum;
 #pragma unroll
           for (int c = 0; c < 64; ++c) v[c] *= inv;
-          store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bs) * p.L + row) * p.H * 64 +
+          store_vec<bf16, 64>(static_cast<bf16*>(p.o) + (size_t(bq) * p.L + row) * p.H * 64 +
                                   size_t(h) * 64, v);
         }
       }

@@ -23,8 +23,10 @@ constexpr int kMaxStreams = 64;                      // video streams per handle
 // device frame counter and read by every later kernel of the frame.
 struct FrameState {
   long long t;          // absolute index of the frame being decoded
-  int slot;             // ring slot that receives this frame: t mod (W+1)
-  int n_valid;          // frames attended to: min(t, W) + 1
+  int slot;             // ring slot that receives this frame: t mod (ring slots)
+  int n_valid;          // frames attended to: min(t, window - 1) + 1
+  int win;              // first ring row (in frames) of the attended keys: 0, or
+                        // for a mirrored ring (slot - n_valid + 1) mod slots
   float2 rope_t[kMaxTemporalPairs];  // (cos, sin) of t * theta^(-2m/d_t), m < d_t/2
 };
 

@@ -45,8 +45,10 @@ constexpr bool epi_normed(int kind) {
 }
 
 struct EpiParams {
-  int M;                 // rows: B video streams x L tokens, row = b L + n
+  int M;                 // rows: n_sub sub-frames x B video streams x L tokens,
+                         // row = (tau B + b) L + n (n_sub = 1: row = b L + n)
   int L;                 // tokens per frame of one stream
+  int B;                 // video streams
   int N;                 // GEMM output columns
   const float* bias;     // [N]
   // RMSNorm row scale (QKV, GELU, FINAL; none when ssq is null)
@@ -64,12 +66,13 @@ struct EpiParams {
   void* kc;              // this block's keys   [B][G][kv_rows][Dh]
   void* vtc;             // this block's values [B][G][Dh][vt_pitch] (transposed)
   int H, G, Dh;
-  int kv_rows;           // (W+1) * M
+  int kv_rows;           // rows of one (stream, group) slab of the ring
   int vt_pitch;          // row pitch of the transposed values (elements)
+  int kv_mirror;         // mirrored ring: rows between a key's two copies (0: one copy)
   const float* gk;       // [Dh] KV-norm gains
   const float* gv;
   int kv_norm;
-  const FrameState* fs;  // stream b's state: fs[b * fs_stride]
+  const FrameState* fs;  // state of stream b, sub-frame tau: fs[b * fs_stride + tau]
   int fs_stride;
   const float2* rope_row;  // [tok_h][d_s/2] (cos, sin)
   const float2* rope_col;  // [tok_w][d_s/2]
@@ -82,8 +85,9 @@ struct EpiParams {
   int out_bf16;          // pixel element type
   int P;                 // pixels per token side
   int tok_h;
-  int pl_mul, pl_add;    // column block c = col / P^2 goes to pixel frame
-                         // c * pl_mul + pl_add of the [C * r_t] output frames
+  int pl_mul, pl_add;    // column block c = col / P^2 of sub-frame tau's row goes
+                         // to pixel frame c * pl_mul + pl_add + tau of the
+                         // [C * r_t] output frames
   // FP8 MLP
   float acc_scale;       // dequantization of the accumulator (1: none)
   float q_inv;           // 1 / static scale of the FP8 output
@@ -207,21 +211,23 @@ __device__ __forceinline__ void rms_head(float* v, const float* g, float eps) {
 
 // Unpatchify / PixelShuffle scatter of 64 finished columns of token `row`:
 // 64 / P output rows of P pixels each; column (b*P + dy)*P + dx maps to pixel
-// frame b*pl_mul + pl_add, pixel row i*P+dy, pixels j*P .. j*P+P-1. The linear
-// head has b = c*r_t + tau (pl_mul 1, pl_add 0); the spatial MLP of sub-frame
-// tau has b = c (pl_mul r_t, pl_add tau). P is a template parameter so the
-// accumulator stays in registers.
+// frame b*pl_mul + pl_add + tau, pixel row i*P+dy, pixels j*P .. j*P+P-1,
+// where tau is the sub-frame of the row (0 unless the launch covers several).
+// The linear head has b = c*r_t + tau (pl_mul 1, pl_add 0); the spatial MLP
+// has b = c (pl_mul r_t; pl_add tau when each sub-frame is its own launch).
+// P is a template parameter so the accumulator stays in registers.
 template <int P>
 __device__ __forceinline__ void pixel_scatter(const EpiParams& p, int row, int col0,
                                               const float* acc) {
-  const int b = row / p.L, n = row - b * p.L;              // stream, token
+  const int bq = row / p.L, n = row - bq * p.L;            // (sub-frame, stream), token
+  const int b = bq % p.B, tau = bq / p.B;
   const int i = n / p.tok_w, j = n - (n / p.tok_w) * p.tok_w;
   const size_t out_w = size_t(p.tok_w) * P;
   const size_t plane = size_t(p.tok_h) * P * out_w;      // one [H][W] pixel frame
 #pragma unroll
   for (int s = 0; s < 64; s += P) {
     const int col = col0 + s;
-    const int ct = (col / (P * P)) * p.pl_mul + p.pl_add;
+    const int ct = (col / (P * P)) * p.pl_mul + p.pl_add + tau;
     const int dy = (col / P) % P;
     const size_t off = size_t(b) * p.out_stride + size_t(ct) * plane +
                        (size_t(i) * P + dy) * out_w + size_t(j) * P;
@@ -345,8 +351,9 @@ __device__ __forceinline__ void qkv_epilogue64(const EpiParams& p, int row, int 
   constexpr int DH = 64;
   const bool valid = row < p.M;
   const int rowc = valid ? row : 0;
-  const int b = rowc / p.L, n = rowc - b * p.L;            // stream, token
-  const FrameState* fs = p.fs + size_t(b) * p.fs_stride;
+  const int bq = rowc / p.L, n = rowc - bq * p.L;          // (sub-frame, stream), token
+  const int b = bq % p.B, tau = bq / p.B;
+  const FrameState* fs = p.fs + size_t(b) * p.fs_stride + tau;
   float* v = acc;
   const int head = col0 / DH;
   scale_bias<DH>(v, rs, p.bias, col0);
@@ -360,18 +367,27 @@ __device__ __forceinline__ void qkv_epilogue64(const EpiParams& p, int row, int 
     if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
     rope_head<DH>(v, n, fs, p);
     const int key = fs->slot * p.L + n;
-    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && b * p.L < p.M, p.status))
+    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key + p.kv_mirror < p.kv_rows && bq * p.L < p.M,
+                              p.status))
       dst = static_cast<bf16*>(p.kc) + ((size_t(b) * p.G + g) * p.kv_rows + key) * DH;
     warp_store_rows64(dst, v, tile, lane);
+    if (p.kv_mirror)                                       // uniform: the second copy
+      warp_store_rows64(dst ? dst + size_t(p.kv_mirror) * DH : nullptr, v, tile, lane);
   } else {                                                 // value group
     const int g = head - p.H - p.G;
     if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
     const int key = fs->slot * p.L + n;
-    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && key < p.vt_pitch && g < p.G &&
-                              b * p.L < p.M, p.status)) {
+    if (valid && FD_IN_BOUNDS(fs->slot >= 0 && key + p.kv_mirror < p.kv_rows &&
+                              key + p.kv_mirror < p.vt_pitch && g < p.G && bq * p.L < p.M,
+                              p.status)) {
       bf16* d = static_cast<bf16*>(p.vtc) + (size_t(b) * p.G + g) * DH * p.vt_pitch + key;
 #pragma unroll
       for (int i = 0; i < DH; ++i) d[size_t(i) * p.vt_pitch] = __float2bfloat16_rn(v[i]);
+      if (p.kv_mirror) {
+#pragma unroll
+        for (int i = 0; i < DH; ++i)
+          d[size_t(i) * p.vt_pitch + p.kv_mirror] = __float2bfloat16_rn(v[i]);
+      }
     }
   }
 }
@@ -381,8 +397,9 @@ template <int KIND, typename T, int DH>
 __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0, float* acc,
                                            float rs) {
   if constexpr (KIND == EPI_QKV) {
-    const int b = row / p.L, n = row - b * p.L;            // stream, token
-    const FrameState* fs = p.fs + size_t(b) * p.fs_stride;
+    const int bq = row / p.L, n = row - bq * p.L;          // (sub-frame, stream), token
+    const int b = bq % p.B, tau = bq / p.B;
+    const FrameState* fs = p.fs + size_t(b) * p.fs_stride + tau;
 #pragma unroll
     for (int hh = 0; hh < 64 / DH; ++hh) {
       float* v = acc + hh * DH;
@@ -398,19 +415,26 @@ __device__ __forceinline__ void epilogue64(const EpiParams& p, int row, int col0
         if (p.kv_norm) rms_head<DH>(v, p.gk, p.eps);
         rope_head<DH>(v, n, fs, p);
         const int key = fs->slot * p.L + n;
-        if (!FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && b * p.L < p.M, p.status)) continue;
+        if (!FD_IN_BOUNDS(fs->slot >= 0 && key + p.kv_mirror < p.kv_rows && bq * p.L < p.M,
+                          p.status))
+          continue;
         T* dst = static_cast<T*>(p.kc) + ((size_t(b) * p.G + g) * p.kv_rows + key) * DH;
         store_vec<T, DH>(dst, v);
+        if (p.kv_mirror) store_vec<T, DH>(dst + size_t(p.kv_mirror) * DH, v);
       } else {                                            // value group
         const int g = head - p.H - p.G;
         if (p.kv_norm) rms_head<DH>(v, p.gv, p.eps);
         const int key = fs->slot * p.L + n;
-        if (!FD_IN_BOUNDS(fs->slot >= 0 && key < p.kv_rows && key < p.vt_pitch && g < p.G &&
-                          b * p.L < p.M, p.status))
+        if (!FD_IN_BOUNDS(fs->slot >= 0 && key + p.kv_mirror < p.kv_rows &&
+                          key + p.kv_mirror < p.vt_pitch && g < p.G && bq * p.L < p.M, p.status))
           continue;
         T* dst = static_cast<T*>(p.vtc) + (size_t(b) * p.G + g) * DH * p.vt_pitch + key;
 #pragma unroll
         for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch] = from_f<T>(v[d]);
+        if (p.kv_mirror) {
+#pragma unroll
+          for (int d = 0; d < DH; ++d) dst[size_t(d) * p.vt_pitch + p.kv_mirror] = from_f<T>(v[d]);
+        }
       }
     }
   } else if constexpr (KIND == EPI_RESID || KIND == EPI_RESID_Q) {

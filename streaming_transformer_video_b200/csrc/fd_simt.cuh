@@ -18,15 +18,24 @@ namespace fd {
 // fs[b (1 + n_sub) + k]:
 //   k = 0: latent frame t = ctr[b] in the backbone ring of W+1 frames;
 //   k = 1 + tau, tau < n_sub (paper head, n_sub = r_t): sub-frame t r_t + tau
-//   in the refinement ring of r_t (W+1) sub-frames (paper Sec. 3.4, Step 2).
-// A frame with absolute index t in a ring of `cap` slots gets slot =
-// t mod cap, n_valid = min(t, cap - 1) + 1, and temporal RoPE angles
-// t * theta^(-2m/d_t) (inv_freq[m], fp64 from the host) reduced mod 2 pi in
-// fp64, so they stay exact for any stream length. One thread per (state,
-// angle); every counter then advances by one. One CTA.
+//   of the refinement ring (paper Sec. 3.4, Step 2), whose window is the last
+//   r_t (W+1) sub-frames.
+// A frame with absolute index t in a ring of `cap` slots and a window of
+// `wnd` frames gets slot = t mod cap, n_valid = min(t, wnd - 1) + 1, and
+// temporal RoPE angles t * theta^(-2m/d_t) (inv_freq[m], fp64 from the host)
+// reduced mod 2 pi in fp64, so they stay exact for any stream length.
+// The refinement ring either has cap = wnd slots (the window is every valid
+// slot, win = 0), or, when all r_t sub-frames of a latent frame go through a
+// refinement block in one launch (sub_mirror = 1), cap = r_t (W+2) - 1 slots
+// stored twice (slot s at frame rows s and s + cap): writing a latent frame's
+// r_t sub-frames then overwrites no slot that an earlier sub-frame of the same
+// frame still attends to, and each sub-frame's window is the contiguous run
+// of rows [win, win + n_valid) with win = (slot - n_valid + 1) mod cap.
+// One thread per (state, angle); every counter then advances by one. One CTA.
 __global__ void __launch_bounds__(256) step_begin_kernel(long long* ctr, FrameState* fs, int W,
                                                          int n_pairs, const double* inv_freq,
-                                                         int n_sub, int B) {
+                                                         int n_sub, int B, int sub_cap,
+                                                         int sub_mirror) {
   __shared__ long long t0[kMaxStreams];
   griddep_wait();
   griddep_launch();
@@ -38,12 +47,16 @@ __global__ void __launch_bounds__(256) step_begin_kernel(long long* ctr, FrameSt
     const int st = i / n_pairs, m = i - st * n_pairs;
     const int b = st / per, k = st - b * per;
     const long long t = k == 0 ? t0[b] : t0[b] * n_sub + (k - 1);
-    const int cap = k == 0 ? W + 1 : n_sub * (W + 1);
+    const int wnd = k == 0 ? W + 1 : n_sub * (W + 1);
+    const int cap = k == 0 ? W + 1 : sub_cap;
     FrameState* f = fs + st;
     if (m == 0) {
+      const int slot = int(t % cap);
+      const int nv = int(t < wnd - 1 ? t : wnd - 1) + 1;
       f->t = t;
-      f->slot = int(t % cap);
-      f->n_valid = int(t < cap - 1 ? t : cap - 1) + 1;
+      f->slot = slot;
+      f->n_valid = nv;
+      f->win = (k > 0 && sub_mirror) ? (slot - nv + 1 + cap) % cap : 0;
     }
     double sn, cs;
     sincos(fmod(double(t) * inv_freq[m], two_pi), &sn, &cs);

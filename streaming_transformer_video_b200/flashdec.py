@@ -34,7 +34,8 @@ EXPORTS = ["fd_create", "fd_reset", "fd_decode_frame", "fd_decode_frame_host", "
            "fd_cache_bytes", "fd_debug_read_slot", "fd_last_step_kernel_ms",
            "fd_selftest_wait_timeout", "fd_mlp_fp8_scales", "fd_debug_block_mlp",
            "fd_reset_stream", "fd_stream_frame_index", "fd_decode_frame_static_scratch",
-           "fd_debug_read_ring", "fd_debug_poison", "fd_debug_set_frame_index"]
+           "fd_debug_read_ring", "fd_debug_poison", "fd_debug_set_frame_index",
+           "fd_debug_ring_layout"]
 
 
 class FDConfigC(ctypes.Structure):
@@ -97,6 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fd_debug_read_ring.argtypes = [vp, i32, i32, i32, i32, _PF]
     lib.fd_debug_poison.argtypes = [vp, i32, vp]
     lib.fd_debug_set_frame_index.argtypes = [vp, i32, i64, vp]
+    lib.fd_debug_ring_layout.argtypes = [vp, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     for name in EXPORTS:
         if name not in ("fd_destroy", "fd_error_string", "fd_last_error"):
             getattr(lib, name).restype = i32
@@ -322,6 +324,14 @@ class FlashDecoder:
         _check(self._lib.fd_debug_read_ring(self.h, block, b, slot, kv, out.ctypes.data_as(_PF)),
                "fd_debug_read_ring")
         return out
+
+    def ring_layout(self, block: int):
+        """(slots, copies) of a block's ring: frame f in slot f mod slots, and
+        with copies == 2 also in slot f mod slots + slots."""
+        n, c = ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(self._lib.fd_debug_ring_layout(self.h, block, ctypes.byref(n), ctypes.byref(c)),
+               "fd_debug_ring_layout")
+        return n.value, c.value
 
     def debug_poison(self, what: int, stream=None):
         """Fill the ring caches with NaN (FD_POISON_RING) and/or the split

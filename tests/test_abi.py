@@ -154,6 +154,7 @@ def test_bad_handle_calls():
     assert lib.fd_debug_read_ring(None, 0, 0, 0, 0, None) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_debug_poison(None, fdb.FD_POISON_RING, None) == fdb.FD_ERR_BAD_HANDLE
     assert lib.fd_debug_set_frame_index(None, 0, 5, None) == fdb.FD_ERR_BAD_HANDLE
+    assert lib.fd_debug_ring_layout(None, 0, ctypes.byref(n), ctypes.byref(n)) == fdb.FD_ERR_BAD_HANDLE
     # a pointer to memory that is not a handle (magic check)
     junk = (ctypes.c_uint32 * 64)()
     assert lib.fd_reset(ctypes.cast(junk, ctypes.c_void_p), None) == fdb.FD_ERR_BAD_HANDLE

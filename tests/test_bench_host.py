@@ -42,9 +42,18 @@ def test_paper_head_flops_count_refinement_windows_and_sub_frames():
     cfg = C["xl_480p_wan22_paper"]
     L, D, H, G, Dh = cfg.L_frm, 1536, 24, 3, 64
     attn = bench.attn_flops_per_launch(cfg)
-    assert len(attn) == 20 + 4 * 2                               # backbone, then r_t x n_refine
+    # bf16, L = 1560 = 8 x 195: all r_t sub-frames of a refinement block in one launch
+    assert bench.refine_batched(cfg)
+    assert len(attn) == 20 + 2                                   # backbone, then n_refine
     assert attn[0] == 4 * L * (2 * L) * H * Dh                     # W = 1: two frames
-    assert attn[-1] == 4 * L * (4 * 2 * L) * H * Dh                # r_t (W+1) = 8 sub-frames
+    assert attn[-1] == 4 * (4 * L * (4 * 2 * L) * H * Dh)          # r_t x (r_t (W+1) = 8 sub-frames)
+    # sub-frame by sub-frame (L not a multiple of 8): r_t x n_refine launches, same total
+    odd = cfg.replace(grid_h=29)
+    assert not bench.refine_batched(odd) and odd.L_frm % 8 != 0
+    attn_odd = bench.attn_flops_per_launch(odd)
+    assert len(attn_odd) == 20 + 4 * 2
+    assert sum(attn_odd[20:]) == 4 * attn_odd[-1] * 2
+    assert not bench.refine_batched(C["tiny_fp32"].replace(head="paper"))   # fp32 path
     k = bench.kind_flops(cfg)
     assert k["qkv"] == 2 * L * D * (H + 2 * G) * Dh
     assert k["upsample"] == 2 * L * D * 4 * D
@@ -54,8 +63,20 @@ def test_paper_head_flops_count_refinement_windows_and_sub_frames():
 def test_kernels_per_frame_counts_the_graph():
     # step_begin, embed, 5 per block, final
     assert bench.kernels_per_frame(C["1080p_wan22"]) == 2 + 5 * 16 + 1 == 83
-    # paper head: upsample, then per sub-frame 5 per refinement block + 2 spatial
-    assert bench.kernels_per_frame(C["xl_480p_wan22_paper"]) == 2 + 5 * 20 + 1 + 4 * (5 * 2 + 2)
+    # paper head: upsample, then 5 per refinement block + 2 spatial, once for all
+    # sub-frames (bf16, L % 8 == 0) or per sub-frame
+    assert bench.kernels_per_frame(C["xl_480p_wan22_paper"]) == 2 + 5 * 20 + 1 + (5 * 2 + 2)
+    assert bench.kernels_per_frame(C["xl_480p_wan22_paper"].replace(grid_h=29)) == \
+        2 + 5 * 20 + 1 + 4 * (5 * 2 + 2)
+    assert bench.kernels_per_frame(C["xl_480p_wan22_paper"].replace(mlp_fp8=1)) == \
+        2 + 6 * 20 + 1 + (6 * 2 + 2)
+
+
+def test_frame_kind_flops_add_up_to_the_frame():
+    for name in ("1080p_wan22", "xl_480p_wan22_paper"):
+        cfg = C[name]
+        total, attn = bench.flops_per_frame(cfg)
+        assert sum(bench.frame_kind_flops(cfg).values()) == total - attn, name
 
 
 def test_batch_scales_work_and_throughput():

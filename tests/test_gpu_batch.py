@@ -66,6 +66,8 @@ def _videos(cfg, B, frames=None):
     small_bf16(batch=2, grid_h=17, grid_w=23, frames=3),                 # 391 tokens per stream
     small_bf16(batch=2, n_heads=8, n_kv_heads=1, d_model=512, frames=3),  # GQA
     small_bf16(batch=2, head="paper", n_refine=2, window=1, frames=3),   # paper head
+    # paper head, 168 tokens: all sub-frames of both streams in one launch per kernel
+    small_bf16(batch=2, head="paper", n_refine=2, window=1, frames=3, grid_h=12, grid_w=14),
 ])
 def test_batched_streams_equal_unbatched_decodes_bit_exact(cfg):
     w = fd_synth.make_weights(cfg)

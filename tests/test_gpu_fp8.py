@@ -75,6 +75,8 @@ def assert_fp8_close(got, ref):
     dict(d_model=512, n_heads=8, n_kv_heads=1, frames=4),       # GQA ratio 8
     dict(d_model=1536, n_heads=24, n_kv_heads=3, n_blocks=1, window=1, frames=3),  # XL block
     dict(head="paper", n_refine=2, window=1, frames=3),         # refinement MLPs in FP8 too
+    # the same with the sub-frames batched (168 tokens)
+    dict(head="paper", n_refine=2, window=1, frames=3, grid_h=12, grid_w=14),
 ])
 def test_small_bf16_fp8_mlp_matches_oracle(kw):
     cfg, w, z = _fp8_case(small_bf16(**kw))
@@ -82,7 +84,8 @@ def test_small_bf16_fp8_mlp_matches_oracle(kw):
 
 
 @pytest.mark.parametrize("fp8", [1, 0])
-@pytest.mark.parametrize("kw", [dict(), dict(head="paper", n_refine=2, window=1)])
+@pytest.mark.parametrize("kw", [dict(), dict(head="paper", n_refine=2, window=1),
+                                dict(head="paper", n_refine=2, window=1, grid_h=12, grid_w=14)])
 def test_block_mlp_on_identical_inputs(fp8, kw):
     # Both sides get the same float32 residual stream x + b_o; the E4M3 codes
     # of its RMSNorm output and of the hidden activation can differ only

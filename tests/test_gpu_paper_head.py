@@ -1,7 +1,14 @@
 """Parity of the CUDA path with the CPU oracle for the paper's output head
 (FlashDecoder paper, Sec. 3.4): temporal upsampling (Eq. 3), refinement
-blocks streaming r_t sub-frames per latent frame through a ring of r_t (W+1)
-sub-frames, RMSNorm + 2-layer spatial MLP + PixelShuffle per sub-frame.
+blocks streaming r_t sub-frames per latent frame, each attending to the last
+r_t (W+1) sub-frames, RMSNorm + 2-layer spatial MLP + PixelShuffle per
+sub-frame.
+
+The bf16 path runs the r_t sub-frames of a latent frame through each
+refinement block in one launch per kernel when L_frm is a multiple of 8
+(a mirrored ring of r_t (W+2) - 1 sub-frames), else one sub-frame at a time;
+both are checked here (BATCHED: 12 x 14 = 168 tokens, two query tiles, the
+second ragged).
 
 Tolerances as for the linear head: fp32 max abs <= 1e-4; bf16 rel L2 <= 2e-2
 and max abs <= 5e-2. Causality, the dependence bound and reset are checked
@@ -21,6 +28,9 @@ TINY_PAPER = fd_synth.CONFIGS["tiny_fp32"].replace(head="paper", n_refine=2)
 
 def small_bf16_paper(**kw):
     return small_bf16(head="paper", n_refine=2).replace(**kw)
+
+
+BATCHED = dict(grid_h=12, grid_w=14)      # 168 tokens, a multiple of 8
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -61,6 +71,16 @@ def test_tiny_fp32_paper_head_matches_oracle(kw):
     # FlashDecoder-XL block shape (D=1536, 24 heads, 3 KV groups) with its
     # two refinement blocks and the W_frm = 2 window
     dict(d_model=1536, n_heads=24, n_kv_heads=3, n_blocks=1, window=1, frames=3),
+    # all sub-frames of a refinement block in one launch
+    dict(BATCHED, frames=5),
+    dict(BATCHED, window=1, frames=7),                      # ring of 11 wraps twice
+    dict(BATCHED, window=0, frames=4),                      # 7 slots, windows of 4
+    dict(BATCHED, r_t=2, window=1, frames=6),
+    dict(BATCHED, r_t=1, frames=4),                         # one sub-frame: W+1 slots, mirrored
+    dict(BATCHED, n_refine=1, frames=4),
+    dict(BATCHED, attn_splits=3, frames=5),                 # split combine over sub-frames
+    dict(grid_h=8, grid_w=16, n_heads=8, n_kv_heads=2, d_model=512, frames=4),   # 128 tokens, GQA
+    dict(BATCHED, d_model=1536, n_heads=24, n_kv_heads=3, n_blocks=1, window=1, frames=3),
 ])
 def test_small_bf16_paper_head_matches_oracle(kw):
     cfg = small_bf16_paper(**kw)
@@ -147,10 +167,12 @@ def test_paper_head_memory_is_constant_over_200_frames():
     dec.close()
 
 
-def test_paper_head_kernel_sequence():
+@pytest.mark.parametrize("batched", [False, True])
+def test_paper_head_kernel_sequence(batched):
     import torch
+    import bench
     from streaming_transformer_video_b200 import FlashDecoder
-    cfg = small_bf16_paper(frames=2)
+    cfg = small_bf16_paper(frames=2, **(BATCHED if batched else {}))
     w = fd_synth.make_weights(cfg)
     z = fd_synth.make_latents(cfg)
     dec = FlashDecoder(cfg, w, kernel_timing=1)
@@ -160,10 +182,36 @@ def test_paper_head_kernel_sequence():
     for t in range(2):
         dec.decode_frame(lat[t], out)
     kinds = [k for k, _ in dec.kernel_ms()]
+    slots, copies = dec.ring_layout(cfg.n_blocks)
     dec.close()
     block = ["qkv", "attn", "oproj", "mlp_up", "mlp_down"]
+    launches = 1 if batched else cfg.r_t          # launches of each refinement kernel
+    assert (copies == 2) == batched == bench.refine_batched(cfg)
     assert kinds == ["step_begin", "embed"] + block * cfg.n_blocks + ["upsample"] + \
-        (block * cfg.n_refine + ["spatial", "final"]) * cfg.r_t
+        (block * cfg.n_refine + ["spatial", "final"]) * launches
+    assert len(kinds) == bench.kernels_per_frame(cfg)
+
+
+@pytest.mark.parametrize("cfg,layout", [
+    (small_bf16_paper(**BATCHED), (4 * 4 - 1, 2)),                 # r_t (W+2) - 1, mirrored
+    (small_bf16_paper(**BATCHED, window=1, r_t=2), (2 * 3 - 1, 2)),
+    (small_bf16_paper(), (4 * 3, 1)),                               # 130 tokens: r_t (W+1)
+    (TINY_PAPER, (TINY_PAPER.r_t * (TINY_PAPER.window + 1), 1)),    # fp32 path
+])
+def test_refinement_ring_layout(cfg, layout):
+    from streaming_transformer_video_b200 import FlashDecoder
+    w = fd_synth.make_weights(cfg)
+    dec = FlashDecoder(cfg, w)
+    try:
+        assert dec.ring_layout(0) == (cfg.window + 1, 1)
+        for l in range(cfg.n_refine):
+            assert dec.ring_layout(cfg.n_blocks + l) == layout
+        # the cache holds every slot and copy
+        kv = 2 * cfg.n_kv_heads * cfg.L_frm * cfg.head_dim * (2 if cfg.dtype == "bf16" else 4)
+        assert dec.cache_bytes() >= (cfg.n_blocks * (cfg.window + 1) +
+                                     cfg.n_refine * layout[0] * layout[1]) * kv
+    finally:
+        dec.close()
 
 
 def test_xl_480p_paper_head_frames_0_to_2_match_oracle():

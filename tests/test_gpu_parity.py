@@ -279,6 +279,7 @@ def test_xl_gqa_480p_full_depth_frames_0_to_2_match_oracle():
     dict(attn_splits=3, grid_h=1, grid_w=1),                  # 1 key tile: empty ranges
     dict(attn_splits=3, n_heads=8, n_kv_heads=1, d_model=512),
     dict(attn_splits=2, head="paper", n_refine=2, window=1, frames=3),
+    dict(attn_splits=4, head="paper", n_refine=1, window=1, frames=3, grid_h=12, grid_w=14),
 ])
 def test_attention_key_splitting_matches_oracle(kw):
     # each (query tile, head) split over several CTAs, partial results

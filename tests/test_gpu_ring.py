@@ -10,7 +10,9 @@ relative to the current window, so videos of any length decode the same way.
 Checked here:
   * slot indexing, exactly: ring slot s of the tcgen05 path (bf16), of every
     video stream of a batch and of the refinement ring holds the frame (or
-    sub-frame) f with f = s mod capacity, post-RoPE at its absolute index;
+    sub-frame) f with f = s mod capacity, post-RoPE at its absolute index; a
+    mirrored refinement ring (all r_t sub-frames through a block in one
+    launch) holds f in both copies, slots s and s + capacity;
   * a ring filled with NaN right after the reset never reaches an output:
     a frame reads only slots written since the reset;
   * a stream restarted after a video whose cache holds NaN decodes its new
@@ -54,20 +56,24 @@ def _rel(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
 
-def _check_ring(cfg, read, candidates, capacity):
-    """read(slot, kv) -> GPU slot [G][L][Dh]; candidates: {index: (k_rot, v)}.
-    Each slot must match exactly the candidate whose index is slot mod
-    capacity, within the value tolerance, and every other one by far less."""
+def _check_ring(cfg, read, candidates, capacity, copies=1):
+    """read(slot, kv) -> GPU slot [G][L][Dh]; candidates: {index: (k_rot, v)},
+    the frames the window attends to. Frame f must sit in slot f mod capacity
+    (and, with two copies, also in that slot + capacity), matching its
+    candidate within the value tolerance and every other one by far less.
+    Without copies the window fills the ring, so every slot is checked."""
     tol = 2e-2 if cfg.dtype == "bf16" else 1e-4
-    assert len(candidates) == capacity
-    for slot in range(capacity):
-        k_gpu, v_gpu = read(slot, 0), read(slot, 1)
-        dist = {f: max(_rel(k_gpu, kr), _rel(v_gpu, vv)) for f, (kr, vv) in candidates.items()}
-        best = min(dist, key=dist.get)
-        assert best % capacity == slot, (slot, dist)
-        assert dist[best] <= tol, (slot, dist)
-        others = [d for f, d in dist.items() if f != best]
-        assert not others or min(others) > 10 * tol, (slot, dist)
+    assert len(candidates) == capacity if copies == 1 else len(candidates) < capacity
+    for f in sorted(candidates):
+        for c in range(copies):
+            slot = f % capacity + c * capacity
+            k_gpu, v_gpu = read(slot, 0), read(slot, 1)
+            dist = {g: max(_rel(k_gpu, kr), _rel(v_gpu, vv)) for g, (kr, vv) in candidates.items()}
+            best = min(dist, key=dist.get)
+            assert best == f, (slot, dist)
+            assert dist[best] <= tol, (slot, dist)
+            others = [d for g, d in dist.items() if g != best]
+            assert not others or min(others) > 10 * tol, (slot, dist)
 
 
 def _backbone_candidates(cfg, ora, l):
@@ -142,6 +148,9 @@ def test_every_stream_of_a_batch_has_its_own_exact_ring():
 
 @pytest.mark.parametrize("cfg", [
     small_bf16(head="paper", n_refine=2, window=1, frames=3),    # 12 sub-frames, 8 slots
+    # 168 tokens: all 4 sub-frames per launch, mirrored ring of 11 slots x 2
+    small_bf16(head="paper", n_refine=2, window=1, frames=4, grid_h=12, grid_w=14),
+    small_bf16(head="paper", n_refine=1, window=2, r_t=2, frames=5, grid_h=12, grid_w=14),
     TINY.replace(head="paper", n_refine=1, window=1, r_t=2, frames=5),   # fp32 path
 ])
 def test_refinement_ring_slots_hold_their_sub_frames_exactly(cfg):
@@ -151,16 +160,19 @@ def test_refinement_ring_slots_hold_their_sub_frames_exactly(cfg):
     ora = oracle.OracleDecoder(cfg, w)
     for t in range(cfg.frames):
         ora.decode_frame(z[t])
-    cap = cfg.r_t * (cfg.window + 1)
+    window = cfg.r_t * (cfg.window + 1)
     try:
         for l in range(cfg.n_refine):
+            cap, copies = dec.ring_layout(cfg.n_blocks + l)
+            assert (cap, copies) in ((window, 1), (cfg.r_t * (cfg.window + 2) - 1, 2))
             subs = ora.refine_window(l)
-            assert subs == list(range(cfg.frames * cfg.r_t - cap, cfg.frames * cfg.r_t))
+            assert subs == list(range(cfg.frames * cfg.r_t - window, cfg.frames * cfg.r_t))
             cand = {}
             for s in subs:
                 k, v = ora.refine_cached_kv(l, s)
                 cand[s] = (_rotated(cfg, k, s), np.stack([v[:, g] for g in range(cfg.n_kv_heads)]))
-            _check_ring(cfg, lambda s, kv: dec.read_ring(cfg.n_blocks + l, 0, s, kv), cand, cap)
+            _check_ring(cfg, lambda s, kv: dec.read_ring(cfg.n_blocks + l, 0, s, kv), cand, cap,
+                        copies)
         # and the backbone ring of the same handle
         for l in range(cfg.n_blocks):
             _check_ring(cfg, lambda s, kv: dec.read_ring(l, 0, s, kv),
@@ -204,6 +216,8 @@ def _decode(cfg, w, videos, poison=False, dec=None):
     small_bf16(window=3, grid_h=17, grid_w=23, frames=6, attn_splits=3),
     small_bf16(batch=2, frames=4),
     small_bf16(head="paper", n_refine=2, window=1, frames=3),        # refinement ring too
+    # mirrored refinement ring (sub-frames batched), two streams
+    small_bf16(head="paper", n_refine=2, window=1, frames=4, grid_h=12, grid_w=14, batch=2),
     TINY.replace(head="paper", n_refine=1, window=1, r_t=2, frames=4),
 ])
 def test_nan_poisoned_ring_never_reaches_outputs(cfg):
@@ -217,10 +231,13 @@ def test_nan_poisoned_ring_never_reaches_outputs(cfg):
     assert_close(cfg, poisoned[0].astype(np.float64), ref)
 
 
-def test_restart_after_a_nan_video_decodes_like_a_fresh_handle():
+@pytest.mark.parametrize("cfg", [
+    small_bf16(batch=2, frames=4),
+    small_bf16(batch=2, frames=4, head="paper", n_refine=1, window=1, grid_h=12, grid_w=14),
+])
+def test_restart_after_a_nan_video_decodes_like_a_fresh_handle(cfg):
     import torch
     from streaming_transformer_video_b200 import FlashDecoder
-    cfg = small_bf16(batch=2, frames=4)
     w = fd_synth.make_weights(cfg)
     v0 = fd_synth.make_latents(cfg, frames=7, seed=1)
     bad = np.full((3,) + v0.shape[1:], np.nan, dtype=np.float32)

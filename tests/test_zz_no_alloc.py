@@ -68,7 +68,11 @@ def test_two_handles_of_different_sizes_take_turns_on_the_array():
     import torch
     from streaming_transformer_video_b200 import FlashDecoder
     cfgs = [small_bf16(attn_splits=2, frames=4),
-            small_bf16(attn_splits=3, grid_h=17, grid_w=23, frames=4)]
+            small_bf16(attn_splits=3, grid_h=17, grid_w=23, frames=4),
+            # two attention launch shapes in one handle: a frame, and all
+            # refinement sub-frames at once (more units on the array)
+            small_bf16(attn_splits=2, head="paper", n_refine=1, window=1, grid_h=12, grid_w=14,
+                       frames=4)]
     ref, fixed, lats, decs = [], [], [], []
     try:
         for cfg in cfgs:
@@ -85,10 +89,10 @@ def test_two_handles_of_different_sizes_take_turns_on_the_array():
             lats.append(lat)
             decs += [a, b]
         for t in range(4):                             # alternate on one stream
-            for i in range(2):
+            for i in range(len(cfgs)):
                 decs[2 * i + 1].decode_frame_static_scratch(lats[i][t], fixed[i][t])
         torch.cuda.synchronize()
-        for i in range(2):
+        for i in range(len(cfgs)):
             assert decs[2 * i + 1].status() == 0
             for t in range(4):
                 np.testing.assert_array_equal(fixed[i][t].float().cpu().numpy(),
