@@ -40,8 +40,8 @@ DEFAULT_CONFIG = "1080p_wan22"
 # profiles/attention_1080p_ncu.md. Keyed by the sha256 of the kernel source:
 # when the kernel changes the figure no longer applies and is reported as null.
 NCU_ATTN_TRAFFIC = {
-    ("1080p_wan22", "18e75f4f177e79c8501a21f412c7d2c45390de89fd1d1f60ae0e490bc18ceb6b"):
-        163831040 + 57682944,
+    ("1080p_wan22", "a862314ce01b65283f2ca9b9c229ab8cc4db5039e586cd1253e84302ff0cb071"):
+        164353536 + 58573312,
 }
 
 
