@@ -67,6 +67,8 @@ class FDConfig:
     batch: int = 1
     # bf16 attention key splitting: 0 = automatic, 1..4 forced
     attn_splits: int = 0
+    # bf16 attention MMA issue: 0 = automatic, 1 = two threads, 2 = one thread
+    attn_issuer: int = 0
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property

@@ -123,6 +123,13 @@ typedef struct {
                             results (1 .. 4); 0 = chosen from the launch's fit
                             to the GPU's CTA slots. Results differ from 1 only
                             by floating-point summation order.               */
+  int32_t attn_issuer;   /* bf16 attention: which threads issue the tensor-core
+                            products of a CTA. 1 = two threads (QK^T and PV
+                            each wait for their own inputs), 2 = one thread
+                            polling both; 0 = one thread for launches with at
+                            least as many CTAs as the GPU has CTA slots, two
+                            otherwise (the faster of the two as measured).
+                            Results are identical bit for bit.               */
 } fd_config;
 
 /*

@@ -19,7 +19,9 @@
 //               S buffer j mod 3 once O += P(j-3) V(j-3) has read that
 //               buffer; lane 1 issues O += P(j) V_j (TS form: P read from
 //               TMEM) as soon as P(j) is written, then releases the K/V stage.
-//               Each lane's tcgen05.commit tracks only its own MMAs.
+//               Each lane's tcgen05.commit tracks only its own MMAs. Launches
+//               with single_issuer set run both streams from lane 0 instead,
+//               polling both hand-offs (same products, same order per stream)
 //   warps 2..5  softmax, one query row per thread: S row from TMEM, base-2
 //               online softmax with lazy rescaling (O is rescaled in TMEM only
 //               when the running max grows by more than 2^8), P packed to bf16
@@ -66,6 +68,7 @@ struct TcAttnParams {
   // bounds of the bounds-checked build (FD_IN_BOUNDS)
   int kv_rows;        // rows of one (layer, stream, group) slab of the ring
   int n_slabs;        // slabs in the ring's tensor maps: layers x B x G
+  int single_issuer;  // 1: one thread issues S and PV (else one lane each)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -234,7 +237,56 @@ __global__ void __launch_bounds__(TcAttnSmem::kThreads, 2)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {                                       // ---- S issuer
+    if (p.single_issuer) {                                 // uniform per launch
+      if (lane == 0) {                                     // ---- one issuer for S and PV
+        // one thread polls both hand-offs, so neither MMA stream waits behind
+        // the other lane's blocking wait in the same warp
+        bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+        int js = 0, jp = 0;                                // next S tile, next PV tile
+        unsigned long long t_idle = 0;
+        while (ok && jp < n_kt) {
+          bool progress = false;
+          if (jp < js && mbar_try_wait(&p_full[jp % 3], (jp / 3) & 1)) {
+            tc_fence_after();
+            const uint32_t sv = smem_u32(smem + S::kKV + (jp % ST) * S::kKVStage + 8192);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_ts(tmem_base + kColO, tmem_base + 64 * (jp % 3) + 8 * k, sw128_desc(sv) + 2 * k,
+                        kIdescO, (jp | k) != 0);
+            tc_commit(&p_free[jp % 3]);
+            tc_commit(&kv_empty[jp % ST]);
+            ++jp;
+            progress = true;
+          }
+          // S(js) once its stage is loaded and O += P(js-3) V(js-3) has read its buffer
+          if (js < n_kt && js < jp + 3 && mbar_try_wait(&kv_full[js % ST], (js / ST) & 1) &&
+              (js < 3 || mbar_try_wait(&p_free[js % 3], ((js / 3) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t sq = smem_u32(smem + S::kQ);
+            const uint32_t sk = smem_u32(smem + S::kKV + (js % ST) * S::kKVStage);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_ss(tmem_base + 64 * (js % 3), sw128_desc(sq) + 2 * k, sw128_desc(sk) + 2 * k,
+                        kIdescS, k != 0);
+            tc_commit(&s_full[js % 3]);
+            ++js;
+            progress = true;
+          }
+          if (progress) {
+            t_idle = 0;
+          } else if (*abort_flag) {
+            ok = false;
+          } else if (t_idle == 0) {
+            t_idle = global_ns();
+          } else if (global_ns() - t_idle > kWaitTimeoutNs) {   // bounded like mbar_wait
+            *abort_flag = 1;
+            report_status(p.status, FD_ERR_TIMEOUT);
+            ok = false;
+          }
+        }
+        if (ok) tc_commit(o_final);
+      }
+    } else if (lane == 0) {                                // ---- S issuer
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       for (int j = 0; ok && j < n_kt; ++j) {
         const int st = j % ST, b = j % 3;

@@ -47,7 +47,7 @@ class FDConfigC(ctypes.Structure):
         ("kernel_timing", ctypes.c_int32), ("head_mode", ctypes.c_int32),
         ("n_refine", ctypes.c_int32), ("mlp_fp8", ctypes.c_int32),
         ("record_mlp_amax", ctypes.c_int32), ("batch", ctypes.c_int32),
-        ("attn_splits", ctypes.c_int32)]
+        ("attn_splits", ctypes.c_int32), ("attn_issuer", ctypes.c_int32)]
 
 
 _PF = ctypes.POINTER(ctypes.c_float)
@@ -162,6 +162,7 @@ def make_config(cfg, io_dtype=None, kernel_timing: bool = False,
     c.record_mlp_amax = int(record_mlp_amax)
     c.batch = int(getattr(cfg, "batch", 1))
     c.attn_splits = int(getattr(cfg, "attn_splits", 0))
+    c.attn_issuer = int(getattr(cfg, "attn_issuer", 0))
     return c
 
 

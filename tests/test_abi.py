@@ -123,6 +123,10 @@ def test_create_rejects_bad_configs_before_touching_the_device():
         c = fdb.make_config(base)
         c.attn_splits = value
         assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
+    for value in (-1, 3):
+        c = fdb.make_config(base)
+        c.attn_issuer = value
+        assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     c = fdb.make_config(bf.replace(mlp_fp8=1), record_mlp_amax=True)
     assert _create(c)[0] == fdb.FD_ERR_INVALID_ARG
     # FP8 without scale pointers: rejected before any device work
@@ -163,14 +167,16 @@ def test_bad_handle_calls():
 
 
 def test_make_config_marshals_every_field():
-    cfg = fd_synth.CONFIGS["xl_720p_wan22_paper"].replace(mlp_fp8=1, batch=3, attn_splits=2)
+    cfg = fd_synth.CONFIGS["xl_720p_wan22_paper"].replace(mlp_fp8=1, batch=3, attn_splits=2,
+                                                          attn_issuer=2)
     c = fdb.make_config(cfg, io_dtype="f32", kernel_timing=2)
     for n in ("latent_ch", "grid_h", "grid_w", "patch", "d_model", "n_heads", "n_kv_heads",
               "head_dim", "n_blocks", "mlp_ratio", "window", "out_ch", "r_t", "px_per_token",
-              "kv_norm", "n_refine", "mlp_fp8", "batch", "attn_splits"):
+              "kv_norm", "n_refine", "mlp_fp8", "batch", "attn_splits", "attn_issuer"):
         assert getattr(c, n) == getattr(cfg, n), n
     assert (c.dtype, c.io_dtype, c.head_mode, c.kernel_timing) == (fdb.FD_BF16, fdb.FD_F32, 1, 2)
     assert c.norm_eps == pytest.approx(cfg.norm_eps) and c.rope_theta == cfg.rope_theta
     assert c.record_mlp_amax == 0
     lin = fdb.make_config(fd_synth.CONFIGS["1080p_wan22"], record_mlp_amax=True)
-    assert (lin.head_mode, lin.n_refine, lin.record_mlp_amax, lin.batch, lin.attn_splits) == (0, 0, 1, 1, 0)
+    assert (lin.head_mode, lin.n_refine, lin.record_mlp_amax, lin.batch, lin.attn_splits,
+            lin.attn_issuer) == (0, 0, 1, 1, 0, 0)

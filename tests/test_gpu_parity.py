@@ -280,6 +280,11 @@ def test_xl_gqa_480p_full_depth_frames_0_to_2_match_oracle():
     dict(attn_splits=3, n_heads=8, n_kv_heads=1, d_model=512),
     dict(attn_splits=2, head="paper", n_refine=2, window=1, frames=3),
     dict(attn_splits=4, head="paper", n_refine=1, window=1, frames=3, grid_h=12, grid_w=14),
+    # one thread issuing both MMA streams (the form large launches take)
+    dict(attn_issuer=2),
+    dict(attn_issuer=2, attn_splits=3, grid_h=1, grid_w=1),   # empty key ranges
+    dict(attn_issuer=2, attn_splits=4, window=3, frames=6),
+    dict(attn_issuer=2, head="paper", n_refine=2, window=1, frames=3, grid_h=12, grid_w=14),
 ])
 def test_attention_key_splitting_matches_oracle(kw):
     # each (query tile, head) split over several CTAs, partial results
@@ -288,6 +293,21 @@ def test_attention_key_splitting_matches_oracle(kw):
     w = fd_synth.make_weights(cfg)
     z = fd_synth.make_latents(cfg)
     assert_close(cfg, gpu_decode(cfg, w, z), oracle_decode(cfg, w, z))
+
+
+@pytest.mark.parametrize("cfg", [
+    small_bf16(attn_splits=2, frames=4),
+    small_bf16(head="paper", n_refine=2, window=1, frames=3, grid_h=12, grid_w=14),
+    # the 480p workload at full width (its launches take two issuing threads)
+    fd_synth.CONFIGS["480p_wan21"].replace(n_blocks=2, frames=4),
+])
+def test_both_mma_issuer_forms_give_identical_bits(cfg):
+    # the same products in the same order per accumulator, whichever threads
+    # issue them
+    w = fd_synth.make_weights(cfg)
+    z = fd_synth.make_latents(cfg)
+    np.testing.assert_array_equal(gpu_decode(cfg.replace(attn_issuer=1), w, z),
+                                  gpu_decode(cfg.replace(attn_issuer=2), w, z))
 
 
 def test_attention_key_splitting_is_deterministic():
