@@ -127,9 +127,10 @@ typedef struct {
                             products of a CTA. 1 = two threads (QK^T and PV
                             each wait for their own inputs), 2 = one thread
                             polling both; 0 = one thread for launches with at
-                            least as many CTAs as the GPU has CTA slots, two
-                            otherwise (the faster of the two as measured).
-                            Results are identical bit for bit.               */
+                            least as many CTAs as the GPU has CTA slots and at
+                            most 100 key tiles of 64 per CTA, two otherwise
+                            (the faster of the two as measured). Results are
+                            identical bit for bit.                           */
 } fd_config;
 
 /*

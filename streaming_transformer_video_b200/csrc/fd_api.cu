@@ -670,11 +670,16 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     ap.kv_rows = io.kv_rows;
     ap.n_slabs = io.n_layers * B * G;
     // one MMA-issuing thread for launches that fill every CTA slot (2 per SM)
-    // at least once; two for under-filled ones (measured: 0.5-3.4% faster
-    // attention at 1080p, 720p and the XL shapes, 2% slower at 480p, which
-    // fills 208 of 296 slots)
+    // at least once with CTAs of at most 100 key tiles (full window); two
+    // otherwise. Measured: 1.5-3.4% faster attention at 720p (56 tiles per
+    // CTA) and for the XL shapes (16-98); 2% slower at 480p (208 CTAs for 296
+    // slots); at 1080p (128-192 tiles) 0.6% fewer cycles per frame but a
+    // 1.2% lower clock under the 1000 W power cap, a net loss
     const long ctas = long((L + 127) / 128) * H * io.n_sub * B * io.n_split;
-    ap.single_issuer = cfg.attn_issuer == 2 || (cfg.attn_issuer == 0 && ctas >= 2L * num_sms);
+    const long window_keys = long(io.kv_mirror ? cfg.r_t * (cfg.window + 1) : io.kv_rows / L) * L;
+    const long tiles = (window_keys + 63) / 64 / io.n_split;
+    ap.single_issuer = cfg.attn_issuer == 2 ||
+                       (cfg.attn_issuer == 0 && ctas >= 2L * num_sms && tiles <= 100);
     // one 128-query tile per CTA, two CTAs per SM (measured faster than two
     // query tiles sharing one CTA, and than three CTAs with single-buffered S)
     using A = TcAttnSmem;
