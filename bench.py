@@ -40,8 +40,8 @@ DEFAULT_CONFIG = "1080p_wan22"
 # profiles/attention_1080p_ncu.md. Keyed by the sha256 of the kernel source:
 # when the kernel changes the figure no longer applies and is reported as null.
 NCU_ATTN_TRAFFIC = {
-    ("1080p_wan22", "a862314ce01b65283f2ca9b9c229ab8cc4db5039e586cd1253e84302ff0cb071"):
-        164353536 + 58573312,
+    ("1080p_wan22", "1034ad4e5f3acab874932dac0e62d5b31664d64097e8713c2afd4bba88c521b3"):
+        163608064 + 58525440,
 }
 
 

@@ -459,6 +459,11 @@ namespace {
 
 bool valid_handle(const fd_handle* h) { return h && h->magic == kMagic; }
 
+// the longest CTA (64-key tiles over a full window) that the automatic
+// choice gives one MMA-issuing thread (measured against 64: the XL paper
+// head's refinement launches, 97 tiles, are 1.2% faster with one thread)
+constexpr long kSingleIssuerMaxTiles = 100;
+
 
 template <int BN, int KIND, bool F8>
 fd_status_t tc_gemm_launch(int M, int N, int num_sms, KernelLaunch* k) {
@@ -679,7 +684,7 @@ fd_status_t fd_handle::add_block(int wi, const BlockIO& io) {
     const long window_keys = long(io.kv_mirror ? cfg.r_t * (cfg.window + 1) : io.kv_rows / L) * L;
     const long tiles = (window_keys + 63) / 64 / io.n_split;
     ap.single_issuer = cfg.attn_issuer == 2 ||
-                       (cfg.attn_issuer == 0 && ctas >= 2L * num_sms && tiles <= 100);
+                       (cfg.attn_issuer == 0 && ctas >= 2L * num_sms && tiles <= kSingleIssuerMaxTiles);
     // one 128-query tile per CTA, two CTAs per SM (measured faster than two
     // query tiles sharing one CTA, and than three CTAs with single-buffered S)
     using A = TcAttnSmem;
